@@ -1,0 +1,95 @@
+"""Planted mistakes in copies of the oracle must each fail at least one pin (no GPU).
+
+A mutant is the oracle module's source with one plausible mistake substituted
+(a dropped term, a wrong sign or index, a transposed layout ...), loaded as a
+fresh module on the CPU.  The real oracle is never modified.
+"""
+
+import importlib.util
+import inspect
+import sys
+import types
+
+import pytest
+
+import oracle.mla_ref as ref
+import oracle.sched_ref as sched
+from oracle_pins import ALL_PINS
+from sched_pins import ALL_SCHED_PINS
+
+ATTN_MUTANTS = {
+    "V is the last 512 columns": ("vals = keys[:, :D_V]", "vals = keys[:, D_K - D_V:]"),
+    "V slice in partials": ("    vals = keys[:, :D_V]\n    qr = q[request]", "    vals = keys[:, 64:]\n    qr = q[request]"),
+    "scale dropped": ("z = scale * (qr[s] @ keys[:n_vis].T)", "z = (qr[s] @ keys[:n_vis].T)"),
+    "lse in log2": ("lse = m + torch.log(zsum)", "lse = (m + torch.log(zsum)) / 0.6931471805599453"),
+    "lse without max": ("lse = m + torch.log(zsum)", "lse = torch.log(zsum)"),
+    "no max subtraction": ("w = torch.exp(z - m[:, None])", "w = torch.exp(z)"),
+    "causal off by one": ("return max(0, int(seqlen) - (s_q - 1 - s))", "return max(0, int(seqlen) - (s_q - s))"),
+    "causal top-left": ("return max(0, int(seqlen) - (s_q - 1 - s))", "return min(int(seqlen), s + 1)"),
+    "page index by modulo": ("page_of_tok = block_table_row.to(torch.int64)[tok // PAGE]",
+                             "page_of_tok = block_table_row.to(torch.int64)[tok % PAGE]"),
+    "slot ignores page offset": ("slot_of_tok = tok % PAGE", "slot_of_tok = tok // PAGE"),
+    "reads the whole last page": [("    if not causal:\n        return int(seqlen)",
+                                   "    if not causal:\n        return -(-int(seqlen) // PAGE) * PAGE"),
+                                  ("tok = torch.arange(seqlen)", "tok = torch.arange(-(-seqlen // PAGE) * PAGE)")],
+    "lse stored [s, h]": ("lse[i, :, s] = l", "lse[i, s % lse.shape[1], :] = l[: lse.shape[2]].sum()"),
+    "empty row lse zero": ("lse = torch.full((len(reqs), h_q, s_q), -math.inf, dtype=_F64)",
+                           "lse = torch.zeros((len(reqs), h_q, s_q), dtype=_F64)"),
+    "merge weights not normalised": ("weights = torch.exp(lses - lse_safe[None])", "weights = torch.exp(lses - m_safe[None])"),
+    "merge lse is max": ("lse = torch.where(finite, m_safe + torch.log(wsum), torch.full_like(m, -math.inf))",
+                         "lse = torch.where(finite, m_safe, torch.full_like(m, -math.inf))"),
+    "partial chunk ignores begin": ("        lo = int(key_begin)\n", "        lo = 0\n"),
+}
+
+SCHED_MUTANTS = {
+    "quota without fixed overhead": ("quota = _ceil_div(total, num_parts) + F if total > 0 else 0",
+                                     "quota = _ceil_div(total, num_parts) if total > 0 else 0"),
+    "total without per-request overhead": ("total = sum(n + F for n in n_blk if n > 0)", "total = sum(n_blk)"),
+    "need without overhead": ("need = (n_blk[r] - k) + F", "need = (n_blk[r] - k)"),
+    "split index not advanced": ("                    split += 1\n", ""),
+    "split takes whole budget": ("t = budget - F", "t = budget"),
+    "block size 128": ("PAGE_BLOCK = 64", "PAGE_BLOCK = 128"),
+    "chunk count ignores earlier splits": ("chunks_so_far += split + 1", "chunks_so_far += 1"),
+}
+
+
+def _mutant(module: types.ModuleType, edits) -> types.ModuleType:
+    """Copy of ``module`` with each (old, new) text substitution applied."""
+    if isinstance(edits, tuple):
+        edits = [edits]
+    mutated = inspect.getsource(module)
+    for old, new in edits:
+        assert mutated.count(old) >= 1, f"mutation anchor not found: {old!r}"
+        mutated = mutated.replace(old, new)
+    name = module.__name__ + "_mutant"
+    spec = importlib.util.spec_from_loader(name, loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__dict__["__name__"] = name
+    sys.modules[name] = mod  # dataclasses / inspect need it registered
+    try:
+        exec(compile(mutated, f"<{name}>", "exec"), mod.__dict__)
+    finally:
+        sys.modules.pop(name, None)
+    return mod
+
+
+def _caught(pins, mod) -> list:
+    failed = []
+    for pin in pins:
+        try:
+            pin(mod)
+        except Exception as e:  # noqa: BLE001 - any failure counts as caught
+            failed.append(f"{pin.__name__}: {type(e).__name__}")
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(ATTN_MUTANTS))
+def test_attention_mutant_is_caught(name):
+    mod = _mutant(ref, ATTN_MUTANTS[name])
+    assert _caught(ALL_PINS, mod), f"mutant '{name}' passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(SCHED_MUTANTS))
+def test_sched_mutant_is_caught(name):
+    mod = _mutant(sched, SCHED_MUTANTS[name])
+    assert _caught(ALL_SCHED_PINS, mod), f"mutant '{name}' passed every pin"
