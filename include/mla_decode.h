@@ -1,0 +1,172 @@
+/*
+ * mla_decode.h -- C ABI of a B200 (sm_100a) paged MLA decode attention library.
+ *
+ * Operation (one latent KV head, "FlashMLA 在 Hopper GPU 上的 MHA 内核调度优化解析",
+ * section 计算边界特性与优化方向抉择): every cached token is one row of d_k = 576
+ * values; it is the key, and its first d_v = 512 values are the value.  For
+ * request b with L_b cached tokens, query row (s, h):
+ *     z_j   = softmax_scale * q[b,s,h,:] . K_j          (j visible)
+ *     out   = sum_j exp(z_j) V_j / sum_j exp(z_j)
+ *     lse   = ln sum_j exp(z_j)
+ * Tokens live in 64-token pages addressed through a block table
+ * ("FlashMLA: 高性能GPU注意力机制计算库" walk-through, section 项目主要功能:
+ * paged KV cache, block size 64, BF16 and FP16).  With causal != 0 and s_q > 1,
+ * query position s (0-based) sees keys j <= L_b - s_q + s (bottom-right
+ * alignment); a row that sees no key gets out = 0 and lse = -inf.
+ *
+ * The work is split across the SMs by a tile scheduler (same walk-through,
+ * section 6. SM资源调度优化; hotdry page section 辅助优化：可编程依赖启动与瓦片调度),
+ * computed by a split-KV kernel, and the pieces of a request that was split are
+ * merged by their log-sum-exp in a combine kernel launched with programmatic
+ * dependent launch (same hotdry section; "DeepSeek开源FlashMLA全解析" 2.1 item 4,
+ * 结果融合).
+ *
+ * Conventions for every call:
+ *  - Pointers named "device" are CUDA device pointers on the current device;
+ *    the caller owns every buffer.  The library allocates and frees nothing on
+ *    these paths and keeps only a per-device cache of SM counts and kernel
+ *    attributes.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *    enqueue work; none synchronises except mla_read_device_status.
+ *  - Return value: MLA_OK (0) or an mla_status code.  Arguments are checked on
+ *    the host before anything is enqueued; a failed check enqueues nothing.
+ *    A failed CUDA launch returns MLA_ERR_CUDA and mla_last_cuda_error() gives
+ *    the cudaError_t (per thread).
+ *  - Device data (lengths, block table) is trusted for shape but bounds-checked
+ *    in the kernels: a page index outside [0, num_pages) is replaced by page 0
+ *    and MLA_DEVERR_PAGE_INDEX is OR-ed into the workspace's error word; a
+ *    pipeline wait that exceeds ~2 s sets MLA_DEVERR_TIMEOUT and the kernel
+ *    returns.  Kernels never trap.
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_HEAD_DIM_K 576
+#define MLA_HEAD_DIM_V 512
+#define MLA_PAGE_SIZE 64
+#define MLA_META_INTS 8
+#define MLA_FIXED_OVERHEAD_BLOCKS 5
+
+#define MLA_DEVERR_TIMEOUT 1
+#define MLA_DEVERR_PAGE_INDEX 2
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer */
+  MLA_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels handle */
+  MLA_ERR_WORKSPACE = 3,   /* workspace smaller than mla_get_workspace_size */
+  MLA_ERR_CUDA = 4         /* a CUDA runtime call failed; see mla_last_cuda_error */
+} mla_status;
+
+typedef enum { MLA_BF16 = 0, MLA_FP16 = 1 } mla_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char* mla_status_string(int status);
+
+/* cudaError_t of the last failed CUDA call made by this thread (0 if none). */
+int mla_last_cuda_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int mla_version(void);
+
+/*
+ * Number of scheduler partitions for `rows` = s_q * h_q query rows per request
+ * on `device` (one partition = one CTA pair per 128-row tile).  Host only; it
+ * queries the device's SM count and cluster occupancy once and caches it.
+ * rows must be in [1, 1024].
+ */
+int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts);
+
+/*
+ * Bytes of workspace mla_decode_fwd needs for this batch, row count and
+ * partition count: a 256-byte error header, then per-chunk fp32 lse partials
+ * [batch + num_sm_parts, rows] and fp32 output partials
+ * [batch + num_sm_parts, rows, 512].  The first 256 bytes must be zero before
+ * the first call (they accumulate device error bits until the caller clears
+ * them).  Host only.
+ */
+int mla_get_workspace_size(int batch, int rows, int num_sm_parts, size_t* bytes);
+
+/*
+ * Tile scheduler ("FlashMLA: 高性能GPU注意力机制计算库", section 6. SM资源调度优化).
+ *   cache_seqlens        device int32 [batch]: cached tokens per request (>= 0)
+ *   batch                1 .. 16384
+ *   rows                 s_q * h_q (used only to validate against num_sm_parts)
+ *   num_sm_parts         from mla_get_num_sm_parts
+ *   tile_sched_metadata  device int32 [num_sm_parts, 8], written: per partition
+ *                        begin_req, begin_block, end_req, end_block (exclusive,
+ *                        lexicographic over (request, 64-token block)),
+ *                        begin_split, 0, 0, 0
+ *   num_splits           device int32 [batch + 1], written: prefix sums of the
+ *                        number of chunks each request is cut into
+ * Blocks n_b = ceil(L_b / 64); quota = ceil(sum_{n_b>0}(n_b + 5) / P) + 5; the
+ * partitions take requests in order and cut a request when its remaining
+ * blocks plus the fixed overhead of 5 exceed what is left of the quota.
+ * Enqueues one single-CTA kernel on `stream`.
+ */
+int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows, int num_sm_parts,
+                     int32_t* tile_sched_metadata, int32_t* num_splits, void* stream);
+
+/*
+ * Decode forward: split-KV kernel, then (programmatic dependent launch) the
+ * log-sum-exp combine kernel.
+ *   q                 device [batch, s_q, h_q, 576], dtype, contiguous, 16-B aligned
+ *   kcache            device [num_pages, 64, 1, 576], dtype, contiguous, 16-B aligned
+ *   num_pages         pages in kcache (>= 1)
+ *   block_table       device int32 [batch, block_table_stride]; entry p of
+ *                     request b is the page holding its tokens 64p .. 64p+63
+ *   block_table_stride  elements between rows of block_table (>= 1)
+ *   cache_seqlens     device int32 [batch], the same values given to mla_get_metadata
+ *   batch, s_q, h_q   s_q * h_q in [1, 1024]
+ *   dtype             MLA_BF16 or MLA_FP16 (q, kcache and out share it)
+ *   softmax_scale     multiplies q.k (finite)
+ *   causal            0 or 1 (see the header comment)
+ *   tile_sched_metadata, num_splits, num_sm_parts   from mla_get_metadata
+ *   workspace         device, >= mla_get_workspace_size bytes, 256-B aligned
+ *   out               device [batch, s_q, h_q, 512], dtype, 16-B aligned (written)
+ *   lse               device fp32 [batch, h_q, s_q] (written; note heads before
+ *                     query positions)
+ * Calls that overlap on the GPU must not share a workspace.
+ */
+int mla_decode_fwd(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                   int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                   int dtype, float softmax_scale, int causal, const int32_t* tile_sched_metadata,
+                   const int32_t* num_splits, int num_sm_parts, void* workspace, size_t workspace_bytes,
+                   void* out, float* lse, void* stream);
+
+/*
+ * The two stages of mla_decode_fwd, exposed for timing and testing; same
+ * arguments and checks.  mla_splitkv_fwd writes out/lse of every request that
+ * was not cut and the partials of the others; mla_combine_fwd merges the
+ * partials (lse = ln sum_c exp(lse_c), out = sum_c exp(lse_c - lse) o_c) and
+ * writes zeros / -inf for requests with no cached token.  mla_combine_fwd uses
+ * programmatic dependent launch, so it may start while the split-KV kernel
+ * drains; it waits for it before reading partials.
+ */
+int mla_splitkv_fwd(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                    int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                    int dtype, float softmax_scale, int causal, const int32_t* tile_sched_metadata,
+                    const int32_t* num_splits, int num_sm_parts, void* workspace, size_t workspace_bytes,
+                    void* out, float* lse, void* stream);
+int mla_combine_fwd(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int dtype,
+                    const int32_t* num_splits, int num_sm_parts, void* workspace, size_t workspace_bytes,
+                    void* out, float* lse, void* stream);
+
+/*
+ * Copy the workspace's error word (MLA_DEVERR_* bits) and the first offending
+ * page index to host `flags[2]`; synchronises `stream`.  Does not clear them.
+ */
+int mla_read_device_status(const void* workspace, void* stream, int32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

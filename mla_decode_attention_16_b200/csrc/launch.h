@@ -1,0 +1,21 @@
+// Host-side launchers of the CUDA path (defined next to each kernel).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+int splitkv_smem_bytes();
+const void* splitkv_kernel_ptr(bool bf16);
+cudaError_t launch_splitkv(bool bf16, const CUtensorMap& qmap, const CUtensorMap& kmap, const DecodeParams& p,
+                           cudaStream_t stream);
+cudaError_t launch_combine(bool bf16, const DecodeParams& p, cudaStream_t stream);
+int metadata_smem_bytes(int batch);
+const void* metadata_kernel_ptr();
+cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta, int32_t* num_splits,
+                            cudaStream_t stream);
+
+}  // namespace mla
