@@ -1,0 +1,419 @@
+"""Benchmark of paged MLA decode on B200 (one JSON line on stdout).
+
+A step is one pass of the whole hot path over one batch: the tile scheduler
+(mla_get_metadata) followed by the decode forward (split-KV kernel + combine
+kernel), inputs resident in HBM.  The default workload is the memory-bound
+decode batch (64 requests x 4096 cached tokens, h_q 16, s_q 1, bf16); pick
+another with --workload.  Throughput uses the pages' cost model:
+bytes = 576*2*sum(L) + q + out + lse, FLOPs = 2*h_q*s_q*(576+512)*sum(L).
+
+Timing: W warm-up steps, then exactly K steps between CUDA events on the
+launching stream, with a barrier and a synchronize on both sides; two resident
+copies of the cache (each larger than the 126 MB L2) alternate between steps so
+no step finds its pages in L2.  Multi-GPU (torchrun): every rank runs its own
+shard of requests (weak scaling, no collective on the data path); the elapsed
+time is the max over ranks.
+
+--impl reference times the CPU oracle (fp64, this host's cores) on a bounded
+sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, algorithmic_cost, make_workload  # noqa: E402
+
+METRIC = "MLA decode TFLOPS & HBM GB/s at 1 B200, % of roofline, vs CPU oracle"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DEFAULT_WORKLOAD = "memory-bound"
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def unit_of(name: str) -> str:
+    w = WORKLOADS[name]
+    return "GB/s" if w.rows < 128 else "TFLOPS"
+
+
+def throughput(cost: dict, seconds: float, unit: str) -> float:
+    if unit == "GB/s":
+        return cost["bytes"] / seconds / 1e9
+    return cost["flops"] / seconds / 1e12
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a scalar over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Seed of rank's shard of requests: rank 0 keeps the workload's own seed."""
+    return base_seed + 7777 * rank
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - NVML missing: report no clocks
+            self.ok = False
+        self.period = period_s
+        self._t = None
+
+    def _sample(self):
+        try:
+            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            fn = getattr(self._nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                self._nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.reasons |= int(fn(self._h))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def profile_traffic(name: str):
+    """DRAM bytes per split-KV launch from the committed ncu summary, if it is for this source."""
+    path = os.path.join(ROOT, "profiles", f"splitkv_{name}.md")
+    src = os.path.join(ROOT, "mla_decode_attention_16_b200", "csrc", "splitkv.cu")
+    try:
+        text = open(path).read()
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m_sha = re.search(r"splitkv\.cu sha256\[:16\]:\s*([0-9a-f]{16})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != digest:
+        return None
+    return float(m_tr.group(1))
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+def oracle_sample(inp, budget_s: float):
+    """Time the fp64 oracle request by request until ~budget_s; returns (seconds, requests)."""
+    import oracle
+
+    done, t0 = [], time.perf_counter()
+    for r in range(inp.batch):
+        oracle.mla_decode_ref(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens, inp.softmax_scale,
+                              inp.causal, requests=[r])
+        done.append(r)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return time.perf_counter() - t0, done
+
+
+def cpu_baseline(inp, name: str, unit: str, budget_s: float):
+    secs, reqs = oracle_sample(inp, budget_s)
+    lens = [int(inp.cache_seqlens[r]) for r in reqs]
+    cost = algorithmic_cost(lens, inp.s_q, inp.h_q)
+    return {"value": throughput(cost, secs, unit), "unit": unit, "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(reqs)} of {inp.batch} requests of the {name} workload, fp64 torch CPU, {secs:.1f} s"}
+
+
+def run_reference(args, name: str):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    unit = unit_of(name)
+    inp = make_workload(name)
+    per_step = max(0.5, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(inp, per_step)
+    vals, secs_tot = [], 0.0
+    for _ in range(args.steps):
+        secs, reqs = oracle_sample(inp, per_step)
+        lens = [int(inp.cache_seqlens[r]) for r in reqs]
+        vals.append(throughput(algorithmic_cost(lens, inp.s_q, inp.h_q), secs, unit))
+        secs_tot += secs
+    value = statistics.median(vals)
+    w = WORKLOADS[name]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs_tot / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(name, world),
+        "cpu_baseline": {"value": value, "unit": unit, "cores": torch.get_num_threads(), "kind": "oracle",
+                         "sample": f"each step: requests of the {w.name} workload until {per_step:.1f} s of "
+                                   f"fp64 CPU work (median over steps)"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(name: str, world: int):
+    w = WORKLOADS[name]
+    return {"workload": name, "description": w.description, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
+            "s_q": w.s_q, "h_q": w.h_q, "d_k": 576, "d_v": 512, "page": 64, "causal": w.causal,
+            "l2": "inputs larger than L2; two resident cache copies alternate between steps",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_gpu(args, name: str):
+    import mla_decode_attention_16_b200 as mla
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    unit = unit_of(name)
+    w = WORKLOADS[name]
+
+    inp = make_workload(name) if rank == 0 else None
+    if rank != 0:
+        import workloads as wl
+        g_inp = wl.make_case  # rank shards differ only by seed; same shapes and length law
+        g = torch.Generator().manual_seed(shard_seed(w.seed, rank))
+        lens = wl.draw_seqlens(w, g)
+        inp = g_inp(w.batch, w.s_q, w.h_q, lens, dtype=w.dtype, std=w.std, causal=w.causal,
+                    seed=shard_seed(w.seed, rank) + 1)
+    lens = [int(x) for x in inp.cache_seqlens.tolist()]
+    cost = algorithmic_cost(lens, inp.s_q, inp.h_q)
+
+    b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
+    rows = s_q * h_q
+    q = inp.q.to(dev)
+    caches = [inp.kcache.to(dev), inp.kcache.to(dev)]
+    bt = inp.block_table.to(dev)
+    sl = inp.cache_seqlens.to(dev)
+    parts = mla.mla_get_num_sm_parts(rows, dev.index)
+    meta = torch.empty(parts, 8, dtype=torch.int32, device=dev)
+    ns = torch.empty(b + 1, dtype=torch.int32, device=dev)
+    ws = mla.alloc_workspace(b, rows, parts, dev)
+    out = torch.empty(b, s_q, h_q, 512, dtype=q.dtype, device=dev)
+    lse = torch.empty(b, h_q, s_q, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        mla.mla_get_metadata(sl, rows, parts, meta, ns, stream=stream)
+        mla.mla_decode_fwd(q, caches[i & 1], bt, sl, inp.softmax_scale, inp.causal, meta, ns, ws, out, lse,
+                           stream=stream)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- warm-up
+    for i in range(args.warmup):
+        step(i)
+    barrier()
+    flags = mla.mla_read_device_status(ws, stream)
+    if flags[0] != 0:
+        raise RuntimeError(f"device error flags {flags}")
+
+    # ---- timed region (device throughput, inputs resident)
+    clocks = ClockSampler(dev.index)
+    est_s = 2e-4 * args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    clocks.start()
+    torch.cuda._sleep(int(min(est_s, 0.5) * 1.0e9))  # head start so the host enqueues ahead of the GPU
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    barrier()
+    clocks.stop()
+    elapsed = ev0.elapsed_time(ev1) / 1000.0
+    elapsed_max = reduce_max(elapsed, dev)
+    value = throughput(cost, elapsed_max / args.steps, unit) * world
+
+    # ---- split-KV kernel alone, CUDA events per launch on the launching stream (roofline)
+    n_prof = max(3, min(args.steps, 200))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_prof)]
+    mla.mla_get_metadata(sl, rows, parts, meta, ns, stream=stream)
+    barrier()
+    torch.cuda._sleep(int(min(2e-4 * n_prof, 0.5) * 1.0e9))
+    for i, (a, z) in enumerate(evs):
+        a.record(stream)
+        mla.mla_splitkv_fwd(q, caches[i & 1], bt, sl, inp.softmax_scale, inp.causal, meta, ns, ws, out, lse,
+                            stream=stream)
+        z.record(stream)
+    barrier()
+    kern_s = statistics.mean(a.elapsed_time(z) for a, z in evs) / 1000.0
+
+    # ---- end to end through the public API with pinned host buffers
+    q_h = inp.q.pin_memory()
+    bt_h = inp.block_table.pin_memory()
+    sl_h = inp.cache_seqlens.pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = q_h.numel() * q_h.element_size() + bt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+    n_e2e = max(3, min(args.steps, 200))
+
+    def e2e_step(i):
+        q.copy_(q_h, non_blocking=True)
+        bt.copy_(bt_h, non_blocking=True)
+        sl.copy_(sl_h, non_blocking=True)
+        step(i)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_e2e):
+        e2e_step(i)
+    e1.record(stream)
+    barrier()
+    e2e_s = reduce_max(e0.elapsed_time(e1) / 1000.0 / n_e2e, dev)
+    e2e_value = throughput(cost, e2e_s, unit) * world
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    if unit == "GB/s":
+        achieved = cost["bytes"] / kern_s / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
+    else:
+        achieved = cost["flops"] / kern_s / 1e12
+        peak = float(peaks["bf16_tflops"])  # fp16 dense tensor rate equals bf16 on this part
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
+    roof["traffic"] = profile_traffic(name)
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["kernel"] = "splitkv_pair_kernel"
+    roof["kernel_us"] = kern_s * 1e6
+    roof["algorithmic_per_launch"] = cost["bytes"] if unit == "GB/s" else cost["flops"]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * elapsed_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if q.dtype == torch.bfloat16 else "fp16",
+        "data": "synthetic", "config": workload_config(name, world),
+        "tflops": cost["flops"] / (elapsed_max / args.steps) / 1e12 * world,
+        "gbps": cost["bytes"] / (elapsed_max / args.steps) / 1e9 * world,
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp, name, unit, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + ["all"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    names = [n for n in WORKLOADS if n != "tiny"] if args.workload == "all" else [args.workload]
+    for name in names:
+        rc = run_reference(args, name) if args.impl == "reference" else run_gpu(args, name)
+        if rc:
+            return rc
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -51,6 +51,7 @@ struct DecodeParams {
   int batch, s_q, h_q, rows, m_tiles, num_parts;
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
+  long long* trace;  // per-block timestamps of CTA 0 (only read by builds with MLA_TRACE)
 };
 
 }  // namespace mla

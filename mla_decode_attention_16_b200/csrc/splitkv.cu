@@ -89,6 +89,24 @@ constexpr uint32_t kColP = 384;  // 2 x 32 columns (16-bit pairs)
 
 __device__ __forceinline__ int box_col(int i, int crank) { return i < 4 ? 256 * crank + 64 * i : 512; }
 
+// The running maximum used as the exponent reference moves only when a new
+// score exceeds it by more than 2^8 (log2 units): the exponentials then stay
+// <= 256 (exact in fp32 and representable in bf16/fp16), O and the row sum are
+// rescaled far less often, and the final out = O / l is unchanged because both
+// always share the same reference.
+constexpr float kRescaleThreshold = 8.0f;
+
+#ifdef MLA_TRACE
+enum TraceEv { kTrProd = 0, kTrQk, kTrPv, kTrSmS, kTrSmX, kTrSmP, kTrNum };
+constexpr int kTrMax = 1024;
+__device__ __forceinline__ void trace(const DecodeParams& p, int ev, uint32_t it) {
+  if (p.trace && blockIdx.x == 0 && it < kTrMax) p.trace[ev * kTrMax + it] = clock64();
+}
+#define MLA_TR(ev, it) trace(p, ev, it)
+#else
+#define MLA_TR(ev, it) ((void)0)
+#endif
+
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   if constexpr (kBF16) {
@@ -176,6 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicCAS(err + 1, 0, page == 0 ? -1 : page);
             page = 0;
           }
+          MLA_TR(kTrProd, it);
           mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
           for (int i = 0; i < kBoxes; ++i)
             tma_load_3d_hint(sbase + kOffK + st * kStageBytes + i * kKBox, &kmap, bar(kKvFull + st),
@@ -196,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (jjp == 0) mbar_wait(bar(kOEmpty), (chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         mbar_wait(bar(kPFull + b), (itp >> 1) & 1, abort_flag, err, kDevErrTimeout);
         tc_fence_after();
+        MLA_TR(kTrPv, itp);
         const uint32_t vbase = sbase + kOffK + st * kStageBytes;
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
           // V rows 16kk..16kk+15: 8-key groups 1024 B apart, 64-column boxes 8 KB apart
@@ -224,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, abort_flag, err, kDevErrTimeout);
           mbar_wait(bar(kSEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
           tc_fence_after();
+          MLA_TR(kTrQk, itc);
           const uint32_t kbase = sbase + kOffK + st * kStageBytes;
           for (int s = 0; s < kQkSteps; ++s) {
             const int box = s < 16 ? s / 4 : 4;
@@ -254,6 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t xfull_remote = mapa(bar(kXFull + q4), peer);
     const uint32_t xempty_remote = mapa(bar(kXEmpty + q4), peer);
     const int sw = lane & 15;
+    // a warp whose 32 rows are all padding (rows >= s_q * h_q) keeps the
+    // barrier protocol but skips the math; its peer warp skips the same way
+    const bool active = mtile * kTileRows + q4 * 32 < R;
     uint32_t it = 0, chunk = 0;
     for (int req = br; req < p.batch && (req < er || (req == er && ek > 0)); ++req) {
       const int L = p.cache_seqlens[req];
@@ -267,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         limit = p.causal ? L - (p.s_q - 1 - row_g / p.h_q) : L;
         limit = limit < 0 ? 0 : limit;
       }
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: row sum relative to it
       for (int jj = 0; jj < nb; ++jj) {
         const uint32_t itc = it + jj;
         const int b = itc & 1;
@@ -275,7 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(bar(kSFull + b), (itc >> 1) & 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();  // reconverge before the warp-collective tcgen05.ld
         tc_fence_after();
-        {
+        if (lane == 0) MLA_TR(kTrSmS, itc);
+        if (active) {
           uint32_t r0[32], r1[32];
           tmem_ld32(t_lane + kColS + 64 * b, r0);
           tmem_ld32(t_lane + kColS + 64 * b + 32, r1);
@@ -289,6 +314,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kSEmpty + b));
+        if (!active) {
+          mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kPFull + b));
+          continue;
+        }
 
         // exchange partial scores with the peer CTA (same rows, other half of the contraction)
         mbar_wait<true>(bar(kXEmpty + q4), (itc & 1) ^ 1, abort_flag, err, kDevErrTimeout);
@@ -311,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           mbar_arrive_expect_tx(bar(kXFull + q4), kXWarp);  // arm the next phase first
           mbar_arrive_cluster(xempty_remote);               // then let the peer send again
+          MLA_TR(kTrSmX, itc);
         }
 
         // online softmax in log2 units
@@ -322,10 +354,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           x[c] = t;
           mx = fmaxf(mx, t);
         }
-        const float m_new = fmaxf(m, mx);
-        const bool resc = (jj > 0) && (m > -INFINITY) && (m_new > m);
-        const float alpha = resc ? ex2(m - m_new) : 1.f;
-        const float base = (m_new == -INFINITY) ? 0.f : m_new;
+        bool resc = false;
+        float alpha = 1.f;
+        if (mx > m + kRescaleThreshold) {  // also true when m is still -inf and a key is visible
+          if (m > -INFINITY) {
+            resc = true;
+            alpha = ex2(m - mx);
+          }
+          m = mx;
+        }
+        const float base = (m == -INFINITY) ? 0.f : m;
         float sum = 0.f;
         uint32_t pk[32];
 #pragma unroll
@@ -336,13 +374,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c2] = pack2<kBF16>(p0, p1);
         }
         l = l * alpha + sum;
-        m = m_new;
 
         mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
         tc_fence_after();
         tmem_st32(t_lane + kColP + 32 * b, pk);
-        if (__any_sync(0xffffffffu, resc)) {
+        if (__any_sync(0xffffffffu, resc && jj > 0)) {
+          // O holds PV of blocks before this one (jj == 0 is overwritten by its own PV)
           mbar_wait(bar(kODone), (itc - 1) & 1, abort_flag, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
@@ -359,52 +397,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kPFull + b));
+        if (lane == 0) {
+          MLA_TR(kTrSmP, itc);
+          mbar_arrive(bar(kPFull + b));
+        }
       }
 
       // epilogue: normalise this CTA's O half and write it
       mbar_wait(bar(kOFinal), chunk & 1, abort_flag, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
-      const bool whole = (lo == 0 && hi == n);
-      const int split_idx = (req == br) ? bs : 0;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const float lse_v = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const int64_t chunk_row = whole ? 0 : (static_cast<int64_t>(p.num_splits[req] + split_idx) * R + row_g);
+      if (active) {
+        const bool whole = (lo == 0 && hi == n);
+        const int split_idx = (req == br) ? bs : 0;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse_v = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        const int64_t chunk_row = whole ? 0 : (static_cast<int64_t>(p.num_splits[req] + split_idx) * R + row_g);
 #pragma unroll 1
-      for (int k = 0; k < 8; ++k) {
-        uint32_t o[32];
-        tmem_ld32(t_lane + kColO + 32 * k, o);
-        tmem_wait_ld();
-        if (row_g < R) {
-          const int col = static_cast<int>(crank) * 256 + 32 * k;
-          if (whole) {
-            uint4* dst = reinterpret_cast<uint4*>(
-                reinterpret_cast<uint16_t*>(p.out) + (static_cast<int64_t>(req) * R + row_g) * kDV + col);
+        for (int k = 0; k < 8; ++k) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + kColO + 32 * k, o);
+          tmem_wait_ld();
+          if (row_g < R) {
+            const int col = static_cast<int>(crank) * 256 + 32 * k;
+            if (whole) {
+              uint4* dst = reinterpret_cast<uint4*>(
+                  reinterpret_cast<uint16_t*>(p.out) + (static_cast<int64_t>(req) * R + row_g) * kDV + col);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack2<kBF16>(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-              w.y = pack2<kBF16>(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-              w.z = pack2<kBF16>(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-              w.w = pack2<kBF16>(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-              dst[v] = w;
+              for (int v = 0; v < 4; ++v) {
+                uint4 w;
+                w.x = pack2<kBF16>(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                w.y = pack2<kBF16>(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                w.z = pack2<kBF16>(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                w.w = pack2<kBF16>(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+                dst[v] = w;
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(p.o_acc + chunk_row * kDV + col);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                     __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
             }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.o_acc + chunk_row * kDV + col);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                   __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
           }
         }
-      }
-      if (crank == 0 && row_g < R) {
-        if (whole) {
-          const int s = row_g / p.h_q, h = row_g % p.h_q;
-          p.lse[static_cast<int64_t>(req) * R + h * p.s_q + s] = lse_v;
-        } else {
-          p.lse_acc[chunk_row] = lse_v;
+        if (crank == 0 && row_g < R) {
+          if (whole) {
+            const int s = row_g / p.h_q, h = row_g % p.h_q;
+            p.lse[static_cast<int64_t>(req) * R + h * p.s_q + s] = lse_v;
+          } else {
+            p.lse_acc[chunk_row] = lse_v;
+          }
         }
       }
       tc_fence_before();
