@@ -160,6 +160,31 @@ int mla_combine_fwd(const int32_t* cache_seqlens, int batch, int s_q, int h_q, i
                     void* out, float* lse, void* stream);
 
 /*
+ * Decode forward for callers that cannot allocate device memory where they
+ * run it -- e.g. a serving loop whose GPU memory is reserved up front by
+ * another allocator, or code that must not call cudaMalloc because it may
+ * synchronise the device -- and so have no workspace to pass.  The pages
+ * describe no counterpart; this is a convenience of this library.
+ * Same arguments, checks and results as mla_decode_fwd, minus the workspace:
+ * the partials go to a 32 MiB scratch array built into the library (every GPU
+ * that loads the library keeps it until the process exits).  Calls needing
+ * more than 32 MiB of workspace (mla_get_workspace_size) return
+ * MLA_ERR_WORKSPACE without launching; allocates nothing (no cudaMalloc,
+ * cudaFree or allocating library call).  The first call on a device looks up
+ * the scratch array's device address (cudaGetSymbolAddress) and caches it;
+ * make that first call before any stream capture.  All calls share the one
+ * scratch array, which keeps the previous call's contents (its error header is
+ * cleared at the start of every call), so calls that may overlap on the GPU --
+ * on different streams, or on the same device from different threads without
+ * ordering -- race and must not be issued.
+ */
+int mla_decode_fwd_static_ws(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                             int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q,
+                             int h_q, int dtype, float softmax_scale, int causal,
+                             const int32_t* tile_sched_metadata, const int32_t* num_splits, int num_sm_parts,
+                             void* out, float* lse, void* stream);
+
+/*
  * Copy the workspace's error word (MLA_DEVERR_* bits) and the first offending
  * page index to host `flags[2]`; synchronises `stream`.  Does not clear them.
  */

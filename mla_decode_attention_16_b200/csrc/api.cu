@@ -220,6 +220,10 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
 
 }  // namespace
 
+namespace mla {
+void set_last_cuda_error(int err) { g_last_cuda_error = err; }
+}  // namespace mla
+
 extern "C" {
 
 const char* mla_status_string(int status) {

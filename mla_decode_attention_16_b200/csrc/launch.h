@@ -17,5 +17,7 @@ int metadata_smem_bytes(int batch);
 const void* metadata_kernel_ptr();
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta, int32_t* num_splits,
                             cudaStream_t stream);
+// Records a cudaError_t for mla_last_cuda_error() (per thread).
+void set_last_cuda_error(int err);
 
 }  // namespace mla
