@@ -106,10 +106,13 @@ int mla_get_workspace_size(int batch, int rows, int num_sm_parts, size_t* bytes)
  *                        begin_split, 0, 0, 0
  *   num_splits           device int32 [batch + 1], written: prefix sums of the
  *                        number of chunks each request is cut into
- * Blocks n_b = ceil(L_b / 64); quota = ceil(sum_{n_b>0}(n_b + 5) / P) + 5; the
- * partitions take requests in order and cut a request when its remaining
- * blocks plus the fixed overhead of 5 exceed what is left of the quota.
- * Enqueues one single-CTA kernel on `stream`.
+ * Blocks n_b = ceil(L_b / 64).  Requests are laid end to end on a line of
+ * units (5 units of fixed overhead, then one unit per block); with the share
+ * S = ceil(sum_{n_b>0}(n_b + 5) / P), partition p owns units [p*S, (p+1)*S),
+ * so its work (blocks + 5 per piece) is at most S + 5, the walk-through's
+ * ceil_div(total, num_sm_parts) + fixed overhead.
+ * Enqueues one single-CTA kernel on `stream` (data-parallel: prefix sums and
+ * one binary search per partition).
  */
 int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows, int num_sm_parts,
                      int32_t* tile_sched_metadata, int32_t* num_splits, void* stream);

@@ -81,8 +81,18 @@ int ensure_device(int device) {
       }
     }
     if (rc != MLA_OK) break;
+    for (int bf = 0; bf < 2 && rc == MLA_OK; ++bf) {
+      for (int np : {16, 32}) {
+        if ((e = cudaFuncSetAttribute(narrow_kernel_ptr(bf == 1, np), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      narrow_smem_bytes(np))) != cudaSuccess) {
+          rc = cuda_fail(e);
+          break;
+        }
+      }
+    }
+    if (rc != MLA_OK) break;
     if ((e = cudaFuncSetAttribute(metadata_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  metadata_smem_bytes(kMaxBatch))) != cudaSuccess) {
+                                  metadata_smem_bytes(kMaxBatch, kMaxParts))) != cudaSuccess) {
       rc = cuda_fail(e);
       break;
     }
@@ -123,10 +133,10 @@ int check_rows(int s_q, int h_q) {
   return MLA_OK;
 }
 
-int encode_2d_q(CUtensorMap* map, const void* q, int64_t rows_total, bool bf16) {
+int encode_2d_q(CUtensorMap* map, const void* q, int64_t rows_total, int box_rows, bool bf16) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDK), static_cast<cuuint64_t>(rows_total)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDK) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kTileRows)};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                         const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -208,13 +218,16 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
   if ((rc = ensure_encode()) != MLA_OK) return rc;
   const bool bf16 = dtype == MLA_BF16;
   CUtensorMap qmap, kmap;
-  if ((rc = encode_2d_q(&qmap, q, static_cast<int64_t>(base.batch) * base.rows, bf16)) != MLA_OK) return rc;
+  const bool narrow = base.rows <= kNarrowMaxRows;
+  if (!narrow &&
+      (rc = encode_2d_q(&qmap, q, static_cast<int64_t>(base.batch) * base.rows, kTileRows, bf16)) != MLA_OK)
+    return rc;
   if ((rc = encode_3d_k(&kmap, kcache, num_pages, bf16)) != MLA_OK) return rc;
   DecodeParams p = base;
   p.block_table = block_table;
   p.block_table_stride = block_table_stride;
   p.num_pages = num_pages;
-  cudaError_t e = launch_splitkv(bf16, qmap, kmap, p, stream);
+  cudaError_t e = narrow ? launch_splitkv_narrow(bf16, q, kmap, p, stream) : launch_splitkv(bf16, qmap, kmap, p, stream);
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
 }
 
@@ -254,6 +267,10 @@ int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts) {
   if (rows > kMaxRows) return MLA_ERR_UNSUPPORTED;
   int rc = ensure_device(device);
   if (rc != MLA_OK) return rc;
+  if (rows <= kNarrowMaxRows) {  // one CTA per SM
+    *num_sm_parts = g_dev[device].sms > 0 ? g_dev[device].sms : 1;
+    return MLA_OK;
+  }
   const int m_tiles = (rows + kTileRows - 1) / kTileRows;
   const int parts = g_dev[device].pairs / m_tiles;
   *num_sm_parts = parts > 0 ? parts : 1;
@@ -271,7 +288,7 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows, int num_
                      int32_t* tile_sched_metadata, int32_t* num_splits, void* stream) {
   if (!cache_seqlens || !tile_sched_metadata || !num_splits) return MLA_ERR_INVALID_ARG;
   if (batch < 1 || rows < 1 || num_sm_parts < 1) return MLA_ERR_INVALID_ARG;
-  if (batch > kMaxBatch || rows > kMaxRows) return MLA_ERR_UNSUPPORTED;
+  if (batch > kMaxBatch || rows > kMaxRows || num_sm_parts > kMaxParts) return MLA_ERR_UNSUPPORTED;
   int dev = 0;
   int rc = current_device(&dev);
   if (rc != MLA_OK) return rc;

@@ -48,11 +48,12 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const DecodeParams
   const int b = blockIdx.y;
   const int row = blockIdx.x * kWarps + warp;
   const int R = p.rows;
-  // num_splits was produced before the split-KV kernel started: safe to read early.
+  // Everything read here (partials, and num_splits from the scheduler two launches back, which the
+  // split-KV kernel itself waited for) is complete and visible once the split-KV grid is.
+  ptx::pdl_wait_primary();
   const int c0 = p.num_splits[b];
   const int nc = p.num_splits[b + 1] - c0;
   if (row >= R || nc == 1) return;
-  ptx::pdl_wait_primary();  // partials are complete and visible after this
 
   const int s = row / p.h_q, h = row % p.h_q;
   const int64_t out_row = (static_cast<int64_t>(b) * R + row) * kDV;

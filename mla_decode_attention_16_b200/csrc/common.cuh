@@ -54,4 +54,16 @@ struct DecodeParams {
   long long* trace;  // per-block timestamps of CTA 0 (only read by builds with MLA_TRACE)
 };
 
+#ifdef MLA_TRACE
+// Developer builds only: per-block clock stamps of CTA 0 into p.trace[event][block].
+enum TraceEv { kTrProd = 0, kTrQk, kTrPv, kTrSmS, kTrSmX, kTrSmP, kTrNum };
+constexpr int kTrMax = 1024;
+__device__ __forceinline__ void trace_stamp(const DecodeParams& p, int ev, uint32_t it) {
+  if (p.trace && blockIdx.x == 0 && it < kTrMax) p.trace[ev * kTrMax + it] = clock64();
+}
+#define MLA_TR(ev, it) trace_stamp(p, ev, it)
+#else
+#define MLA_TR(ev, it) ((void)0)
+#endif
+
 }  // namespace mla

@@ -12,8 +12,16 @@ int splitkv_smem_bytes();
 const void* splitkv_kernel_ptr(bool bf16);
 cudaError_t launch_splitkv(bool bf16, const CUtensorMap& qmap, const CUtensorMap& kmap, const DecodeParams& p,
                            cudaStream_t stream);
+// Few-row kernel (s_q * h_q <= kNarrowMaxRows): one CTA per partition.
+constexpr int kNarrowMaxRows = 32;
+int narrow_rows_padded(int rows);
+int narrow_smem_bytes(int np);
+const void* narrow_kernel_ptr(bool bf16, int np);
+cudaError_t launch_splitkv_narrow(bool bf16, const void* q, const CUtensorMap& kmap, const DecodeParams& p,
+                                  cudaStream_t stream);
 cudaError_t launch_combine(bool bf16, const DecodeParams& p, cudaStream_t stream);
-int metadata_smem_bytes(int batch);
+int metadata_smem_bytes(int batch, int num_parts);
+constexpr int kMaxParts = 1024;  // partitions the metadata kernel stages in shared memory
 const void* metadata_kernel_ptr();
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta, int32_t* num_splits,
                             cudaStream_t stream);

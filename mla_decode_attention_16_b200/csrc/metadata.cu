@@ -1,84 +1,134 @@
 // Tile scheduler ("FlashMLA: 高性能GPU注意力机制计算库", section 6. SM资源调度优化;
 // "FlashMLA 在 Hopper GPU 上的 MHA 内核调度优化解析", 辅助优化：可编程依赖启动与瓦片调度).
 //
-// Every request is n_b = ceil(L_b / 64) blocks of 64 tokens and each piece of
-// a request costs a fixed overhead F = 5 blocks (loading Q, filling the
-// pipeline, writing partials, merging).  The num_sm_parts partitions each get
-// quota = ceil(sum_{n_b > 0}(n_b + F) / num_sm_parts) + F and take requests in
-// order; a request whose remaining blocks plus F exceed what is left of the
-// quota is cut (the partition takes left - F blocks if that is positive) and
-// continues in the next partition.  The last partition takes whatever is left.
+// Every request is n_b = ceil(L_b / 64) blocks of 64 tokens, and each piece of
+// work on a request costs a fixed overhead of F = 5 blocks (Q load, pipeline
+// fill, epilogue, merge).  The requests are laid end to end on a line of
+// units -- F overhead units, then one unit per block -- and partition p of P
+// owns the units [p*S, (p+1)*S) with the share S = ceil(total / P), so block k
+// of request b belongs to partition (cum_b + F + k) / S.  A partition's work is
+// its blocks plus F per piece; only its first piece can have its overhead
+// units in the previous partition, so the work is at most S + F, which is the
+// pages' per-partition quota ceil_div(total, num_sm_parts) + fixed overhead.
 //
-// One CTA: the lengths are staged in shared memory with coalesced loads, the
-// total is a block reduction, then one thread walks the requests (a few cycles
-// per request) and writes the [num_sm_parts, 8] table and the [batch + 1]
-// chunk-count prefix sums.
+// Everything is data-parallel (one CTA of 1024 threads): two block-wide
+// prefix sums (units per request, pieces per request) and one binary search
+// per partition boundary, instead of a walk whose length grows with
+// batch + partitions.
 #include "common.cuh"
 #include "launch.h"
 
 namespace mla {
 namespace metadata {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+
+// Exclusive prefix sum over v[0..n) in place (block-wide, all threads call it); returns the total.
+template <typename T>
+__device__ long long block_exclusive_scan(T* v, int n, long long* warp_tot) {
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int lo = min(n, t * per), hi = min(n, lo + per);
+  long long s = 0;
+  for (int i = lo; i < hi; ++i) s += v[i];
+  long long incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    long long wt = warp_tot[lane];
+    long long wi = wt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    warp_tot[lane] = wi - wt;  // exclusive offset of each warp
+    if (lane == 31) warp_tot[kWarps] = wi;
+  }
+  __syncthreads();
+  long long run = warp_tot[w] + incl - s;
+  for (int i = lo; i < hi; ++i) {
+    const long long x = v[i];
+    v[i] = static_cast<T>(run);
+    run += x;
+  }
+  const long long total = warp_tot[kWarps];
+  __syncthreads();
+  return total;
+}
 
 __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                             int num_parts, int32_t* __restrict__ meta,
                                                             int32_t* __restrict__ num_splits) {
-  extern __shared__ int s_blocks[];
-  __shared__ long long s_partial[kThreads / 32];
-  long long local = 0;
+  // smem: unit offset of each request (cum, int64) [batch + 1], then blocks / pieces per request (int32)
+  extern __shared__ long long s_dyn[];
+  long long* s_cum = s_dyn;
+  int* s_cnt = reinterpret_cast<int*>(s_dyn + batch + 1);
+  __shared__ long long s_warp[kWarps + 1];
+  // the split-KV kernel that follows may start its prologue now; it waits for this grid before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   for (int i = threadIdx.x; i < batch; i += kThreads) {
     const int L = seqlens[i];
-    const int n = L > 0 ? (L + kPage - 1) / kPage : 0;
-    s_blocks[i] = n;
-    if (n > 0) local += n + kFixedOverhead;
+    const int n = L > 0 ? L / kPage + (L % kPage != 0) : 0;
+    s_cum[i] = n > 0 ? static_cast<long long>(n) + kFixedOverhead : 0;
+    s_cnt[i] = n;  // blocks, replaced by pieces below
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-  if ((threadIdx.x & 31) == 0) s_partial[threadIdx.x >> 5] = local;
   __syncthreads();
-  if (threadIdx.x != 0) return;
+  const long long total = block_exclusive_scan(s_cum, batch, s_warp);
+  const long long share = total > 0 ? (total + num_parts - 1) / num_parts : 0;
 
-  long long total = 0;
-  for (int w = 0; w < kThreads / 32; ++w) total += s_partial[w];
-  const long long quota = total > 0 ? (total + num_parts - 1) / num_parts + kFixedOverhead : 0;
-
-  int r = 0, k = 0, split = 0, chunks = 0;
-  num_splits[0] = 0;
-  for (int part = 0; part < num_parts; ++part) {
-    const int begin_r = r, begin_k = k, begin_split = split;
-    long long left = quota;
-    const bool last = part == num_parts - 1;
-    while (r < batch) {
-      const int n = s_blocks[r];
-      if (n == 0) {
-        num_splits[r + 1] = chunks;
-        ++r;
-        continue;
-      }
-      const long long need = static_cast<long long>(n - k) + kFixedOverhead;
-      if (need <= left || last) {
-        left -= need;
-        chunks += split + 1;
-        num_splits[r + 1] = chunks;
-        ++r;
-        k = 0;
-        split = 0;
-      } else {
-        const long long take = left - kFixedOverhead;
-        if (take > 0) {
-          k += static_cast<int>(take);
-          ++split;
-        }
-        break;
-      }
+  for (int i = threadIdx.x; i < batch; i += kThreads) {
+    const long long n = s_cnt[i];
+    long long pieces = 0;
+    if (n > 0) {
+      const long long first = s_cum[i] + kFixedOverhead;  // unit of block 0
+      pieces = (first + n - 1) / share - first / share + 1;
     }
+    s_cnt[i] = static_cast<int>(pieces);
+  }
+  __syncthreads();
+  const long long total_pieces = block_exclusive_scan(s_cnt, batch, s_warp);
+  for (int i = threadIdx.x; i < batch; i += kThreads) num_splits[i] = s_cnt[i];
+  if (threadIdx.x == 0) num_splits[batch] = static_cast<int32_t>(total_pieces);
+
+  // partition boundaries: unit x -> (last request with cum <= x, blocks of it before x), or (batch, 0)
+  auto locate = [&](long long x, int& r, int& k) {
+    if (share == 0 || x >= total) {
+      r = batch;
+      k = 0;
+      return;
+    }
+    int lo = 0, hi = batch - 1;  // largest r with s_cum[r] <= x (s_cum[0] = 0 <= x)
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_cum[mid] <= x)
+        lo = mid;
+      else
+        hi = mid - 1;
+    }
+    r = lo;
+    const long long off = x - s_cum[lo] - kFixedOverhead;
+    k = off > 0 ? static_cast<int>(off) : 0;
+  };
+  for (int part = threadIdx.x; part < num_parts; part += kThreads) {
+    int br, bk, er, ek;
+    locate(static_cast<long long>(part) * share, br, bk);
+    locate(static_cast<long long>(part + 1) * share, er, ek);
+    int bsplit = 0;
+    if (bk > 0) bsplit = part - static_cast<int>((s_cum[br] + kFixedOverhead) / share);
     int32_t* row = meta + part * kMetaInts;
-    row[0] = begin_r;
-    row[1] = begin_k;
-    row[2] = r;
-    row[3] = k;
-    row[4] = begin_split;
+    row[0] = br;
+    row[1] = bk;
+    row[2] = er;
+    row[3] = ek;
+    row[4] = bsplit;
     row[5] = 0;
     row[6] = 0;
     row[7] = 0;
@@ -87,13 +137,16 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
 
 }  // namespace metadata
 
-int metadata_smem_bytes(int batch) { return batch * static_cast<int>(sizeof(int)); }
+int metadata_smem_bytes(int batch, int num_parts) {
+  (void)num_parts;
+  return (batch + 1) * static_cast<int>(sizeof(long long) + sizeof(int));
+}
 const void* metadata_kernel_ptr() { return reinterpret_cast<const void*>(&metadata::metadata_kernel); }
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta, int32_t* num_splits,
                             cudaStream_t stream) {
-  metadata::metadata_kernel<<<1, metadata::kThreads, metadata_smem_bytes(batch), stream>>>(seqlens, batch, num_parts,
-                                                                                            meta, num_splits);
+  metadata::metadata_kernel<<<1, metadata::kThreads, metadata_smem_bytes(batch, num_parts), stream>>>(
+      seqlens, batch, num_parts, meta, num_splits);
   return cudaGetLastError();
 }
 

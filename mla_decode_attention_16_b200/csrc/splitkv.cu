@@ -96,16 +96,7 @@ __device__ __forceinline__ int box_col(int i, int crank) { return i < 4 ? 256 * 
 // always share the same reference.
 constexpr float kRescaleThreshold = 8.0f;
 
-#ifdef MLA_TRACE
-enum TraceEv { kTrProd = 0, kTrQk, kTrPv, kTrSmS, kTrSmX, kTrSmP, kTrNum };
-constexpr int kTrMax = 1024;
-__device__ __forceinline__ void trace(const DecodeParams& p, int ev, uint32_t it) {
-  if (p.trace && blockIdx.x == 0 && it < kTrMax) p.trace[ev * kTrMax + it] = clock64();
-}
-#define MLA_TR(ev, it) trace(p, ev, it)
-#else
-#define MLA_TR(ev, it) ((void)0)
-#endif
+
 
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -161,6 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // launched as a programmatic dependent of the previous kernel in the stream (normally the
+  // scheduler): everything above overlapped it; nothing it wrote is read before this wait
+  pdl_wait_primary();
   if (threadIdx.x == 0) pdl_launch_dependents();
 
   const int br = meta[0], bk = meta[1], er = meta[2], ek = meta[3], bs = meta[4];
@@ -485,13 +479,15 @@ cudaError_t launch_splitkv(bool bf16, const CUtensorMap& qmap, const CUtensorMap
   cfg.blockDim = dim3(splitkv::kThreads);
   cfg.dynamicSmemBytes = splitkv::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (bf16) return cudaLaunchKernelEx(&cfg, splitkv::splitkv_pair_kernel<true>, qmap, kmap, p);
   return cudaLaunchKernelEx(&cfg, splitkv::splitkv_pair_kernel<false>, qmap, kmap, p);
 }

@@ -1,0 +1,540 @@
+// Split-KV MLA decode kernel for requests with few query rows (s_q * h_q <= 32).
+//
+// Same computation as the pair kernel (splitkv.cu): per chunk of 64-token
+// pages, scores, online softmax ("FlashMLA 在 Hopper GPU 上的 MHA 内核调度优化解析",
+// 跷跷板调度的数学重构: rescaled accumulation equals the plain softmax), PV,
+// and out/lse or fp32 partials for the combine (辅助优化：可编程依赖启动与瓦片调度).
+//
+// With <= 32 query rows the decode is bound by HBM (the cost model of
+// 计算边界特性与优化方向抉择: intensity ~ 2 * h_q * s_q FLOP/B), so the goal is
+// to stream pages at full bandwidth with one CTA per SM and no traffic between
+// SMs.  A 128 x 512 fp32 output would not fit TMEM next to the scores, so the
+// value product is computed transposed:
+//   S   [rows x 64 keys] = Q . K^T      (M = 128 lanes, A = Q resident in TMEM,
+//                                        B = the page's key box in smem)
+//   O^T [512 x rows]   += V^T . P^T     (4 tiles of M = 128 d_v rows, N = NP;
+//                                        A = MN-major view of the page's first
+//                                        8 column boxes, B = P row-major in smem)
+// TMEM: O^T (two buffers of 4*NP columns when NP = 16, one when NP = 32),
+// S 64 columns, Q 288 columns (576 16-bit values per row).  Q of even chunks
+// lives in lane quadrant 0 and of odd chunks in quadrant 1, so the next
+// chunk's Q is written while the current chunk runs (the MMA computes all 128
+// lanes; rows outside the current quadrant are ignored).
+//
+// Roles (384 threads): warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0
+// issues every tcgen05.mma; warps 4-7: warp 4 + (chunk & 1) runs the softmax
+// of a chunk (one thread per query row) and all four rescale O^T when a row's
+// exponent reference moves; warps 8-11 write each chunk's epilogue from its
+// O^T buffer while the next chunk runs, and warps 8 / 9 load Q for even / odd
+// chunks.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace mla {
+namespace narrow {
+
+using namespace ptx;
+
+constexpr int kThreads = 384;
+constexpr int kBoxes = kDK / 64;              // 9 column boxes of 64 columns (128 B)
+constexpr int kKBox = kPage * 128;            // 8 KB: one page x 64 columns
+constexpr int kStageBytes = kBoxes * kKBox;   // 72 KB: one page
+constexpr int kStages = 3;
+constexpr int kQCols = kDK / 2;               // 288 TMEM columns of packed 16-bit pairs
+constexpr float kRescaleThreshold = 8.0f;     // see splitkv.cu
+
+enum Bar {
+  kKvFull = 0,
+  kKvEmpty = kKvFull + kStages,
+  kQFull = kKvEmpty + kStages,  // [2] Q rows of a chunk parity written to TMEM
+  kQEmpty = kQFull + 2,         // [2] last Q.K^T of a chunk of that parity completed
+  kSFull = kQEmpty + 2,
+  kSEmpty,
+  kPFull,                       // [2]
+  kPEmpty = kPFull + 2,         // [2]
+  kODone = kPEmpty + 2,         // one phase per PV
+  kOFinal,                      // [2] one phase per chunk using that O^T buffer
+  kOEmpty = kOFinal + 2,        // [2] epilogue finished reading that O^T buffer
+  kStats = kOEmpty + 2,         // [2] row sums / reference maxima of a chunk parity in smem
+  kDrain = kStats + 2,
+  kNumBars
+};
+
+template <int NP>
+struct Layout {
+  static constexpr int kOBufs = NP == 16 ? 2 : 1;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffP = kOffK + kStages * kStageBytes;  // 1024-aligned
+  static constexpr int kPBytes = NP * 128;                     // P: NP rows x 64 keys (16-bit)
+  static constexpr int kOffRed = kOffP + 2 * kPBytes;
+  // floats: alpha [2][NP], flag [2], row sums [2][NP], reference max [2][NP]
+  static constexpr int kRedFloats = 2 * NP + 2 + 2 * NP + 2 * NP;
+  static constexpr int kOffBar = (kOffRed + kRedFloats * 4 + 7) / 8 * 8;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = kOBufs * 4 * NP;
+  static constexpr uint32_t kColQ = kColS + kPage;
+  static_assert(kColQ + kQCols <= kTmemCols, "TMEM budget");
+};
+
+template <bool kBF16>
+__device__ __forceinline__ void store_out(void* out, int64_t idx, float v) {
+  if constexpr (kBF16)
+    reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<__half*>(out)[idx] = __float2half_rn(v);
+}
+
+template <bool kBF16>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  if constexpr (kBF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+template <int NP>
+__device__ __forceinline__ void tmem_ld_np(uint32_t taddr, uint32_t (&r)[NP]) {
+  if constexpr (NP == 16)
+    tmem_ld16(taddr, r);
+  else
+    tmem_ld32(taddr, r);
+}
+template <int NP>
+__device__ __forceinline__ void tmem_st_np(uint32_t taddr, const uint32_t (&r)[NP]) {
+  if constexpr (NP == 16)
+    tmem_st16(taddr, r);
+  else
+    tmem_st32(taddr, r);
+}
+
+// One chunk of a partition: blocks [lo, hi) of request req (n blocks in all).
+struct Chunk {
+  int req, lo, hi, n, L, split;
+};
+
+// Next non-empty chunk at or after request `req` of the partition (req advanced past it).
+__device__ __forceinline__ bool next_chunk(const DecodeParams& p, int br, int bk, int er, int ek, int bs, int& req,
+                                           Chunk& c) {
+  for (; req < p.batch && (req < er || (req == er && ek > 0)); ++req) {
+    const int L = p.cache_seqlens[req];
+    const int n = (L + kPage - 1) / kPage;
+    const int lo = (req == br) ? bk : 0;
+    const int hi = (req == er) ? ek : n;
+    if (hi <= lo) continue;
+    c = Chunk{req, lo, hi, n, L, req == br ? bs : 0};
+    ++req;
+    return true;
+  }
+  return false;
+}
+
+template <bool kBF16, int NP>
+__global__ void __launch_bounds__(kThreads, 1)
+    splitkv_narrow_kernel(const void* __restrict__ qptr, const __grid_constant__ CUtensorMap kmap,
+                          const DecodeParams p) {
+  using Lay = Layout<NP>;
+  constexpr int kOBufs = Lay::kOBufs;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::kOffBar + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
+  float* s_alpha = reinterpret_cast<float*>(smem + Lay::kOffRed);          // [2][NP]
+  volatile int* s_flag = reinterpret_cast<volatile int*>(s_alpha + 2 * NP);  // [2]
+  float* s_lsum = s_alpha + 2 * NP + 2;                                   // [2][NP]
+  float* s_mref = s_lsum + 2 * NP;                                        // [2][NP]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int part = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool four = i == kPFull || i == kPFull + 1 || i == kOEmpty || i == kOEmpty + 1;
+      mbar_init(bar(i), four ? 4u : 1u);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 64) prefetch_tmap(&kmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // launched as a programmatic dependent of the previous kernel in the stream (normally the
+  // scheduler): the prologue above overlapped it; nothing it wrote is read before this wait
+  pdl_wait_primary();
+  if (threadIdx.x == 0) pdl_launch_dependents();
+
+  const int* meta = p.meta + part * kMetaInts;
+  const int br = meta[0], bk = meta[1], er = meta[2], ek = meta[3], bs = meta[4];
+  const int R = p.rows;
+  int* err = p.err;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (pages only)
+    if (lane == 0) {
+      const uint64_t evict_first = policy_evict_first();
+      uint32_t it = 0;
+      int cur = br;
+      Chunk ch;
+      while (!*abort_flag && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
+        const int32_t* bt = p.block_table + static_cast<int64_t>(ch.req) * p.block_table_stride;
+        for (int blk = ch.lo; blk < ch.hi; ++blk, ++it) {
+          if (*abort_flag) break;
+          const int st = it % kStages;
+          mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          int page = bt[blk];
+          if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
+            atomicOr(err, kDevErrPage);
+            atomicCAS(err + 1, 0, page == 0 ? -1 : page);
+            page = 0;
+          }
+          MLA_TR(kTrProd, it);
+          mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
+          for (int i = 0; i < kBoxes; ++i)
+            tma_load_3d_hint(sbase + Lay::kOffK + st * kStageBytes + i * kKBox, &kmap, bar(kKvFull + st), 64 * i,
+                             0, page, evict_first);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, kPage, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, NP, true, false);
+      uint32_t it = 0, chunk = 0;
+      auto issue_pv = [&](uint32_t itp, int jjp, bool last) {
+        const int st = itp % kStages;
+        const int b = itp & 1;
+        const int ob = chunk % kOBufs;
+        if (jjp == 0) mbar_wait(bar(kOEmpty + ob), ((chunk / kOBufs) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kPFull + b), (itp >> 1) & 1, abort_flag, err, kDevErrTimeout);
+        tc_fence_after();
+        MLA_TR(kTrPv, itp);
+        const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
+        const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
+        const uint32_t dcol = tmem + ob * 4 * NP;
+#pragma unroll 1
+        for (int m = 0; m < 4; ++m) {
+          for (int kk = 0; kk < kPage / 16; ++kk) {
+            // V^T rows m*128 .. m*128+127 = column boxes 2m, 2m+1 (8 KB apart); keys 16kk .. 16kk+15
+            const uint64_t adesc = smem_desc_sw128(kst + (2 * m) * kKBox + kk * 2048, kKBox, 1024);
+            const uint64_t bdesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
+            umma_ss(dcol + m * NP, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(bar(kKvEmpty + st));
+        umma_commit(bar(kPEmpty + b));
+        umma_commit(bar(kODone));
+        if (last) umma_commit(bar(kOFinal + ob));
+      };
+      int cur = br;
+      Chunk ch;
+      while (!*abort_flag && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
+        const int nb = ch.hi - ch.lo;
+        const int qpar = chunk & 1;
+        mbar_wait(bar(kQFull + qpar), (chunk >> 1) & 1, abort_flag, err, kDevErrTimeout);
+        tc_fence_after();
+        for (int jj = 0; jj < nb; ++jj) {
+          const uint32_t itc = it + jj;
+          const int st = itc % kStages;
+          mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          tc_fence_after();
+          MLA_TR(kTrQk, itc);
+          const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
+#pragma unroll 1
+          for (int i = 0; i < kBoxes; ++i) {
+            for (int kk = 0; kk < 4; ++kk) {
+              const int s = 4 * i + kk;
+              const uint64_t bdesc = smem_desc_sw128(kst + i * kKBox + kk * 32, 16, 1024);
+              umma_ts(tmem + Lay::kColS, tmem + Lay::kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(bar(kSFull));
+          if (jj == nb - 1) umma_commit(bar(kQEmpty + qpar));
+          if (jj > 0) issue_pv(itc - 1, jj - 1, false);
+        }
+        issue_pv(it + nb - 1, nb - 1, true);
+        it += nb;
+        ++chunk;
+      }
+      umma_commit(bar(kDrain));
+      mbar_wait_drain(bar(kDrain), 0);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax (one warp per chunk) + O^T rescale
+    const int q4 = warp & 3;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int r = lane;
+    uint32_t it = 0, chunk = 0;
+    int cur = br;
+    Chunk ch;
+    while (next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
+      const int nb = ch.hi - ch.lo;
+      const int par = chunk & 1;
+      const bool smx = q4 == par;  // warp 4 for even chunks, warp 5 for odd ones (lane quadrant = parity)
+      const int ob = chunk % kOBufs;
+      int limit = 0;
+      if (smx && r < R) {
+        limit = p.causal ? ch.L - (p.s_q - 1 - r / p.h_q) : ch.L;
+        limit = limit < 0 ? 0 : limit;
+      }
+      float m = -INFINITY, l = 0.f;
+      for (int jj = 0; jj < nb; ++jj) {
+        const uint32_t itc = it + jj;
+        const int b = itc & 1;
+        if (smx) {
+          mbar_wait(bar(kSFull), itc & 1, abort_flag, err, kDevErrTimeout);
+          __syncwarp();
+          tc_fence_after();
+          if (lane == 0) MLA_TR(kTrSmS, itc);
+          float x[64];
+          {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(t_lane + Lay::kColS, r0);
+            tmem_ld32(t_lane + Lay::kColS + 32, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              x[c] = __uint_as_float(r0[c]);
+              x[32 + c] = __uint_as_float(r1[c]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kSEmpty));
+
+          const int kbase = (ch.lo + jj) * kPage;
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float t = (kbase + c < limit) ? x[c] * p.scale_log2 : -INFINITY;
+            x[c] = t;
+            mx = fmaxf(mx, t);
+          }
+          bool resc = false;
+          float alpha = 1.f;
+          if (mx > m + kRescaleThreshold) {
+            if (m > -INFINITY && jj > 0) {
+              resc = true;
+              alpha = ex2(m - mx);
+            }
+            m = mx;
+          }
+          const float base = (m == -INFINITY) ? 0.f : m;
+          float sum = 0.f;
+          uint32_t pk[32];
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const float p0 = ex2(x[2 * c2] - base);
+            const float p1 = ex2(x[2 * c2 + 1] - base);
+            sum += p0 + p1;
+            pk[c2] = pack2<kBF16>(p0, p1);
+          }
+          l = l * alpha + sum;
+          const bool any_resc = __any_sync(0xffffffffu, resc);
+          if (r < NP) s_alpha[b * NP + r] = alpha;
+          if (lane == 0) s_flag[b] = any_resc ? 1 : 0;
+          mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          if (r < NP) {
+            // P row r: 64 keys = 128 bytes, 16-byte chunks XOR-swizzled by row (128-byte swizzle)
+            uint8_t* prow = smem + Lay::kOffP + b * Lay::kPBytes + r * 128;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              *reinterpret_cast<uint4*>(prow + ((k ^ (r & 7)) << 4)) =
+                  make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          }
+          fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+          if (lane == 0) MLA_TR(kTrSmP, itc);
+        }
+        named_bar_sync(1, 128);
+        if (s_flag[b] && jj > 0) {
+          mbar_wait(bar(kODone), (itc - 1) & 1, abort_flag, err, kDevErrTimeout);
+          __syncwarp();
+          tc_fence_after();
+#pragma unroll 1
+          for (int mt = 0; mt < 4; ++mt) {
+            uint32_t o[NP];
+            const uint32_t col = ob * 4 * NP + mt * NP;
+            tmem_ld_np<NP>(t_lane + col, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < NP; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * s_alpha[b * NP + c]);
+            tmem_st_np<NP>(t_lane + col, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kPFull + b));
+      }
+      if (smx) {
+        // this stats slot was last used by chunk - 2; with two O^T buffers its epilogue may still
+        // be reading it (with one buffer the MMA order already guarantees it finished)
+        if (kOBufs == 2 && chunk >= 2)
+          mbar_wait(bar(kOEmpty + par), ((chunk >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        if (r < NP) {
+          s_lsum[par * NP + r] = l;
+          s_mref[par * NP + r] = m;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kStats + par));
+      }
+      it += nb;
+      ++chunk;
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ Q loads (warps 8 / 9) and epilogue (8-11)
+    const int q4 = warp & 3;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int r = lane;
+    auto load_q = [&](const Chunk& c, uint32_t idx) {
+      // Q rows of chunk idx into lane quadrant idx & 1 (this warp's quadrant)
+      mbar_wait(bar(kQEmpty + (idx & 1)), ((idx >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+      __syncwarp();
+      tc_fence_after();
+      const uint4* qrow = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint16_t*>(qptr) + (static_cast<int64_t>(c.req) * R + (r < R ? r : 0)) * kDK);
+#pragma unroll 1
+      for (int c32 = 0; c32 < kQCols / 32; ++c32) {
+        uint32_t w[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 d = make_uint4(0, 0, 0, 0);
+          if (r < R) d = __ldg(qrow + c32 * 8 + v);
+          w[4 * v] = d.x;
+          w[4 * v + 1] = d.y;
+          w[4 * v + 2] = d.z;
+          w[4 * v + 3] = d.w;
+        }
+        tmem_st32(t_lane + Lay::kColQ + 32 * c32, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kQFull + (idx & 1)));
+    };
+    auto epilogue = [&](const Chunk& c, uint32_t idx) {
+      const int ob = idx % kOBufs;
+      const int par = idx & 1;
+      mbar_wait(bar(kOFinal + ob), (idx / kOBufs) & 1, abort_flag, err, kDevErrTimeout);
+      mbar_wait(bar(kStats + par), (idx >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      __syncwarp();
+      tc_fence_after();
+      const bool whole = (c.lo == 0 && c.hi == c.n);
+      const int64_t chunk0 = whole ? 0 : static_cast<int64_t>(p.num_splits[c.req] + c.split) * R;
+      const float* ls = s_lsum + par * NP;
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        uint32_t o[NP];
+        tmem_ld_np<NP>(t_lane + ob * 4 * NP + mt * NP, o);
+        tmem_wait_ld();
+        const int d = mt * 128 + q4 * 32 + lane;
+#pragma unroll
+        for (int cc = 0; cc < NP; ++cc) {
+          if (cc < R) {
+            const float lc = ls[cc];
+            const float v = lc > 0.f ? __uint_as_float(o[cc]) / lc : 0.f;
+            if (whole)
+              store_out<kBF16>(p.out, (static_cast<int64_t>(c.req) * R + cc) * kDV + d, v);
+            else
+              p.o_acc[(chunk0 + cc) * kDV + d] = v;
+          }
+        }
+      }
+      if (q4 == 0 && r < R) {
+        const float lr = ls[r];
+        const float lse_v = lr > 0.f ? (s_mref[par * NP + r] + log2f(lr)) * 0.69314718055994531f : -INFINITY;
+        if (whole) {
+          const int s = r / p.h_q, h = r % p.h_q;
+          p.lse[static_cast<int64_t>(c.req) * R + h * p.s_q + s] = lse_v;
+        } else {
+          p.lse_acc[chunk0 + r] = lse_v;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kOEmpty + ob));
+    };
+    int cur = br;
+    Chunk ch, nx;
+    bool have = next_chunk(p, br, bk, er, ek, bs, cur, ch);
+    if (have && q4 == 0) load_q(ch, 0);
+    uint32_t chunk = 0;
+    while (have) {
+      const bool more = next_chunk(p, br, bk, er, ek, bs, cur, nx);
+      if (more && q4 == static_cast<int>((chunk + 1) & 1)) load_q(nx, chunk + 1);  // overlaps this chunk
+      epilogue(ch, chunk);
+      ch = nx;
+      have = more;
+      ++chunk;
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+template <int NP>
+const void* kernel_ptr(bool bf16) {
+  return bf16 ? reinterpret_cast<const void*>(&splitkv_narrow_kernel<true, NP>)
+              : reinterpret_cast<const void*>(&splitkv_narrow_kernel<false, NP>);
+}
+
+}  // namespace narrow
+
+int narrow_rows_padded(int rows) { return rows <= 16 ? 16 : 32; }
+
+int narrow_smem_bytes(int np) {
+  return np == 16 ? narrow::Layout<16>::kSmemBytes : narrow::Layout<32>::kSmemBytes;
+}
+
+const void* narrow_kernel_ptr(bool bf16, int np) {
+  return np == 16 ? narrow::kernel_ptr<16>(bf16) : narrow::kernel_ptr<32>(bf16);
+}
+
+cudaError_t launch_splitkv_narrow(bool bf16, const void* q, const CUtensorMap& kmap, const DecodeParams& p,
+                                  cudaStream_t stream) {
+  const int np = narrow_rows_padded(p.rows);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_parts);
+  cfg.blockDim = dim3(narrow::kThreads);
+  cfg.dynamicSmemBytes = narrow_smem_bytes(np);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (np == 16) {
+    if (bf16) return cudaLaunchKernelEx(&cfg, narrow::splitkv_narrow_kernel<true, 16>, q, kmap, p);
+    return cudaLaunchKernelEx(&cfg, narrow::splitkv_narrow_kernel<false, 16>, q, kmap, p);
+  }
+  if (bf16) return cudaLaunchKernelEx(&cfg, narrow::splitkv_narrow_kernel<true, 32>, q, kmap, p);
+  return cudaLaunchKernelEx(&cfg, narrow::splitkv_narrow_kernel<false, 32>, q, kmap, p);
+}
+
+}  // namespace mla

@@ -18,7 +18,7 @@ def _ceil_div(a, b):
 
 
 def check_schedule(sched, seqlens, num_parts, F=5):
-    """Invariants any valid output must satisfy (independent of the walk's details)."""
+    """Invariants any valid output must satisfy (independent of how it was computed)."""
     meta, num_splits = sched.tile_schedule_ref(seqlens, num_parts, F)
     b = len(seqlens)
     n = [_ceil_div(L, 64) for L in seqlens]
@@ -28,24 +28,30 @@ def check_schedule(sched, seqlens, num_parts, F=5):
     covered = {}
     split_seen = {r: [] for r in range(b)}
     total = sum(x + F for x in n if x > 0)
-    quota = _ceil_div(total, num_parts) + F if total else 0
+    share = _ceil_div(total, num_parts) if total else 0
     prev_end = (0, 0)
     for p, m in enumerate(meta):
-        assert (m[0], m[1]) == prev_end, f"part {p} does not start where part {p - 1} ended"
+        if p == 0:
+            first = next((r for r in range(b) if n[r] > 0), b)
+            assert (m[0], m[1]) == (first, 0), f"part 0 begins at {(m[0], m[1])}"
+        else:
+            assert (m[0], m[1]) == prev_end, f"part {p} does not start where part {p - 1} ended"
         assert (m[0], m[1]) <= (m[2], m[3]), f"part {p} ends before it begins"
         prev_end = (m[2], m[3])
         chunks = sched.chunks_of_part(m, seqlens)
-        cost = 0
+        load = 0
         for (r, lo, hi, si) in chunks:
             assert 0 <= lo < hi <= n[r]
             for k in range(lo, hi):
                 assert (r, k) not in covered, f"block {(r, k)} covered twice"
                 covered[(r, k)] = p
             split_seen[r].append(si)
-            cost += (hi - lo) + F
-        if p < num_parts - 1 and total:
-            assert cost <= quota, f"part {p} cost {cost} above quota {quota}"
-    assert prev_end == (b, 0), f"walk did not finish: ended at {prev_end}"
+            load += (hi - lo) + F
+        if total:
+            assert load <= share + F, f"part {p} load {load} above share + F = {share + F}"
+            if (p + 1) * share <= total:
+                assert load >= share - F, f"part {p} load {load} below share - F = {share - F}"
+    assert prev_end == (b, 0), f"partitions do not end at (b, 0): {prev_end}"
     for r in range(b):
         for k in range(n[r]):
             assert (r, k) in covered, f"block {(r, k)} not covered"
@@ -83,16 +89,14 @@ def pin_sched_invariants_random(sched):
 
 
 def pin_sched_balance(sched):
-    """Equal requests over equal parts: every part but the last carries at least quota - 2F."""
+    """Equal requests: every partition's work (blocks + F per chunk) is within F of the share."""
     lens = [4096] * 128
     P = 74
     meta, _ = sched.tile_schedule_ref(lens, P, 5)
-    total = 128 * (64 + 5)
-    quota = _ceil_div(total, P) + 5
-    for p in range(P - 1):
-        chunks = sched.chunks_of_part(meta[p], lens)
-        cost = sum(hi - lo + 5 for (_, lo, hi, _) in chunks)
-        assert quota - 10 <= cost <= quota, (p, cost, quota)
+    share = _ceil_div(128 * (64 + 5), P)
+    loads = [sum(hi - lo + 5 for (_, lo, hi, _) in sched.chunks_of_part(meta[p], lens)) for p in range(P)]
+    assert all(share - 5 <= x <= share + 5 for x in loads[:-1]), loads
+    assert sum(x - 5 * len(sched.chunks_of_part(meta[p], lens)) for p, x in enumerate(loads)) == 128 * 64
 
 
 ALL_SCHED_PINS = [pin_sched_golden, pin_sched_invariants_edges, pin_sched_invariants_random, pin_sched_balance]

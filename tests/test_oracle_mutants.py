@@ -42,14 +42,19 @@ ATTN_MUTANTS = {
 }
 
 SCHED_MUTANTS = {
-    "quota without fixed overhead": ("quota = _ceil_div(total, num_parts) + F if total > 0 else 0",
-                                     "quota = _ceil_div(total, num_parts) if total > 0 else 0"),
-    "total without per-request overhead": ("total = sum(n + F for n in n_blk if n > 0)", "total = sum(n_blk)"),
-    "need without overhead": ("need = (n_blk[r] - k) + F", "need = (n_blk[r] - k)"),
-    "split index not advanced": ("                    split += 1\n", ""),
-    "split takes whole budget": ("t = budget - F", "t = budget"),
+    "share rounded down": ("share = _ceil_div(total, num_parts) if total > 0 else 0",
+                           "share = max(1, total // num_parts) if total > 0 else 0"),
+    "share without per-request overhead": ("total = sum(F + n for n in n_blk if n > 0)", "total = sum(n_blk)"),
+    "no overhead units on the line": ("        x += F  # the request's overhead units\n", ""),
+    "overhead after the blocks": [("        x += F  # the request's overhead units\n", ""),
+                                  ("            x += 1\n", "            x += 1\n        x += F\n")],
     "block size 128": ("PAGE_BLOCK = 64", "PAGE_BLOCK = 128"),
-    "chunk count ignores earlier splits": ("chunks_so_far += split + 1", "chunks_so_far += 1"),
+    "split index not recorded": ("chunks.append((part, r, lo, k, per_req.get(r, 0)))", "chunks.append((part, r, lo, k, 0))"),
+    "begin split dropped": ("first_of_part[part] = (r, lo, si if lo > 0 else 0)", "first_of_part[part] = (r, lo, 0)"),
+    "chunk count off by one": ("num_splits[r + 1] = num_splits[r] + per_req.get(r, 0)",
+                               "num_splits[r + 1] = num_splits[r] + per_req.get(r, 0) + (r == 0)"),
+    "empty partitions end at (b, 0)": ("            nxt = first_of_part[p]\n        begins[p] = nxt",
+                                       "            nxt = first_of_part[p]\n        begins[p] = nxt if p in first_of_part else (b, 0, 0)"),
 }
 
 
