@@ -39,15 +39,20 @@ def _inputs():
     return [f for f in files if f.endswith((".cu", ".cuh", ".h"))]
 
 
+FLAGS_RECORD = LIB + ".flags"  # extra flags of the library in place (developer builds add some)
+
+
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
+    if os.path.exists(FLAGS_RECORD) and open(FLAGS_RECORD).read().strip():
+        return True  # the library in place is a developer build
     t = os.path.getmtime(LIB)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
 def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str = LIB) -> str:
-    if not force and out == LIB and not needs_build():
+    if not force and out == LIB and not extra_flags and not needs_build():
         return LIB
     tmp = out + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC,
@@ -58,6 +63,9 @@ def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str =
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     os.replace(tmp, out)
+    if out == LIB:
+        with open(FLAGS_RECORD, "w") as f:
+            f.write(" ".join(extra_flags))
     return out
 
 

@@ -98,7 +98,7 @@ int ensure_device(int device) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * 512);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(splitkv_threads());
     cfg.dynamicSmemBytes = splitkv_smem_bytes();
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -133,14 +133,17 @@ int check_rows(int s_q, int h_q) {
   return MLA_OK;
 }
 
-int encode_2d_q(CUtensorMap* map, const void* q, int64_t rows_total, int box_rows, bool bf16) {
+// Box of box_cols x box_rows elements of q viewed as [rows_total, 576]; box_cols * 2 bytes must
+// equal the swizzle span (64 columns with 128-byte swizzle, 32 with 64-byte swizzle).
+int encode_2d_q(CUtensorMap* map, const void* q, int64_t rows_total, int box_rows, int box_cols,
+                CUtensorMapSwizzle swizzle, bool bf16) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDK), static_cast<cuuint64_t>(rows_total)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kDK) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                         const_cast<void*>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     g_last_cuda_error = static_cast<int>(r);
@@ -149,15 +152,17 @@ int encode_2d_q(CUtensorMap* map, const void* q, int64_t rows_total, int box_row
   return MLA_OK;
 }
 
-int encode_3d_k(CUtensorMap* map, const void* kc, int64_t num_pages, bool bf16) {
+// Box of box_cols columns x one 64-token page of the cache viewed as [pages, 64, 576].
+int encode_3d_k(CUtensorMap* map, const void* kc, int64_t num_pages, int box_cols, CUtensorMapSwizzle swizzle,
+                bool bf16) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDK), static_cast<cuuint64_t>(kPage),
                               static_cast<cuuint64_t>(num_pages)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDK) * 2, static_cast<cuuint64_t>(kDK) * 2 * kPage};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kPage), 1};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kPage), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
                         const_cast<void*>(kc), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     g_last_cuda_error = static_cast<int>(r);
@@ -217,17 +222,20 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
   if ((rc = ensure_device(dev)) != MLA_OK) return rc;
   if ((rc = ensure_encode()) != MLA_OK) return rc;
   const bool bf16 = dtype == MLA_BF16;
-  CUtensorMap qmap, kmap;
+  CUtensorMap qrmap, kmap, krmap;
   const bool narrow = base.rows <= kNarrowMaxRows;
-  if (!narrow &&
-      (rc = encode_2d_q(&qmap, q, static_cast<int64_t>(base.batch) * base.rows, kTileRows, bf16)) != MLA_OK)
-    return rc;
-  if ((rc = encode_3d_k(&kmap, kcache, num_pages, bf16)) != MLA_OK) return rc;
+  if ((rc = encode_3d_k(&kmap, kcache, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf16)) != MLA_OK) return rc;
+  if (!narrow) {  // the pair kernel also takes 32-column boxes of the columns 512..575 of q and of the cache
+    if ((rc = encode_2d_q(&qrmap, q, static_cast<int64_t>(base.batch) * base.rows, kTileRows, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B, bf16)) != MLA_OK)
+      return rc;
+    if ((rc = encode_3d_k(&krmap, kcache, num_pages, 32, CU_TENSOR_MAP_SWIZZLE_64B, bf16)) != MLA_OK) return rc;
+  }
   DecodeParams p = base;
   p.block_table = block_table;
   p.block_table_stride = block_table_stride;
   p.num_pages = num_pages;
-  cudaError_t e = narrow ? launch_splitkv_narrow(bf16, q, kmap, p, stream) : launch_splitkv(bf16, qmap, kmap, p, stream);
+  cudaError_t e = narrow ? launch_splitkv_narrow(bf16, q, kmap, p, stream) : launch_splitkv(bf16, q, qrmap, kmap, krmap, p, stream);
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
 }
 

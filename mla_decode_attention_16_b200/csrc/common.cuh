@@ -54,12 +54,13 @@ struct DecodeParams {
   long long* trace;  // per-block timestamps of CTA 0 (only read by builds with MLA_TRACE)
 };
 
-#ifdef MLA_TRACE
-// Developer builds only: per-block clock stamps of CTA 0 into p.trace[event][block].
-enum TraceEv { kTrProd = 0, kTrQk, kTrPv, kTrSmS, kTrSmX, kTrSmP, kTrNum };
+// Developer trace events (stamped only by builds with MLA_TRACE).
+enum TraceEv { kTrProd = 0, kTrQk, kTrPv, kTrSmS, kTrSmX, kTrSmP, kTrSend, kTrSmC, kTrA, kTrB, kTrC, kTrD, kTrE, kTrF, kTrG, kTrH, kTrNum };
 constexpr int kTrMax = 1024;
+#ifdef MLA_TRACE
+// Per-block clock stamps of CTAs 0 and 1 into p.trace[cta][event][block].
 __device__ __forceinline__ void trace_stamp(const DecodeParams& p, int ev, uint32_t it) {
-  if (p.trace && blockIdx.x == 0 && it < kTrMax) p.trace[ev * kTrMax + it] = clock64();
+  if (p.trace && blockIdx.x < 2 && it < kTrMax) p.trace[(blockIdx.x * kTrNum + ev) * kTrMax + it] = clock64();
 }
 #define MLA_TR(ev, it) trace_stamp(p, ev, it)
 #else

@@ -9,9 +9,12 @@
 namespace mla {
 
 int splitkv_smem_bytes();
+int splitkv_threads();
 const void* splitkv_kernel_ptr(bool bf16);
-cudaError_t launch_splitkv(bool bf16, const CUtensorMap& qmap, const CUtensorMap& kmap, const DecodeParams& p,
-                           cudaStream_t stream);
+// qrmap: 32-column boxes (64-byte swizzle) of q's columns 512..575; kmap: 64-column boxes (128-byte
+// swizzle) of the cache; krmap: 32-column boxes (64-byte swizzle) of the cache.
+cudaError_t launch_splitkv(bool bf16, const void* q, const CUtensorMap& qrmap, const CUtensorMap& kmap,
+                           const CUtensorMap& krmap, const DecodeParams& p, cudaStream_t stream);
 // Few-row kernel (s_q * h_q <= kNarrowMaxRows): one CTA per partition.
 constexpr int kNarrowMaxRows = 32;
 int narrow_rows_padded(int rows);

@@ -37,6 +37,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
+// Relaxed arrive on a peer CTA's mbarrier.  `dep` is an input of the instruction, so it issues only
+// after dep was computed, and so after every load dep was computed from has completed.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed_after(uint32_t remote_bar, float dep) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar), "f"(dep)
+               : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -63,19 +69,23 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 
 // Bounded wait for the phase of parity `parity` to complete.
 // Returns false (after flagging) on timeout or when the CTA already aborted.
+// The abort flag and the clock are looked at only every 16 polls, so a waiting
+// warp issues little besides the polls themselves.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int* err_word, int err_code) {
-  if (*abort_flag) return false;
   if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  if (*abort_flag) return false;
   const long long t0 = clock64();
-  while (true) {
+  for (uint32_t n = 1;; ++n) {
     if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
-      *abort_flag = 1;
-      if (err_word) atomicOr(err_word, err_code);
-      return false;
+    if ((n & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kWaitCycles) {
+        *abort_flag = 1;
+        if (err_word) atomicOr(err_word, err_code);
+        return false;
+      }
     }
   }
 }
@@ -115,6 +125,10 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void* tmap,
       : "memory");
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* gptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(gptr)));
+}
+
 // ----------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -139,6 +153,22 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remot
       "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)), "r"(__float_as_uint(d)),
       "r"(remote_bar)
       : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to a peer
+// CTA's shared memory; completes `bytes` on the peer's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src_cta), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk copy of this thread has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- PDL
@@ -235,6 +265,23 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ----------------------------------------------------------------- math
+// 24-bit packing of fp32 values: the top three bytes of four floats in three
+// words (sign, exponent and 15 mantissa bits; relative error below 2^-15 after
+// unpacking, which re-inserts a half step for the dropped byte).
+__device__ __forceinline__ void pack24(uint32_t a, uint32_t b, uint32_t c, uint32_t d, uint32_t& w0, uint32_t& w1,
+                                       uint32_t& w2) {
+  w0 = __byte_perm(a, b, 0x5321);
+  w1 = __byte_perm(b, c, 0x6532);
+  w2 = __byte_perm(c, d, 0x7653);
+}
+__device__ __forceinline__ void unpack24(uint32_t w0, uint32_t w1, uint32_t w2, float& a, float& b, float& c,
+                                         float& d) {
+  a = __uint_as_float((w0 << 8) | 0x80u);
+  b = __uint_as_float((__byte_perm(w0, w1, 0x5430) & 0xFFFFFF00u) | 0x80u);
+  c = __uint_as_float((__byte_perm(w1, w2, 0x4320) & 0xFFFFFF00u) | 0x80u);
+  d = __uint_as_float((w2 & 0xFFFFFF00u) | 0x80u);
+}
+
 // Warp-wide maximum of a float (sm_100a redux).
 __device__ __forceinline__ float warp_max(float x) {
   float y;
@@ -264,6 +311,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr, uint32_t
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
+// Same with 64-byte swizzling (mode 4): K-major rows of 64 bytes, 8-row atoms of 512 bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;
   return d;
 }
 

@@ -1,4 +1,4 @@
-// Split-KV MLA decode kernel for sm_100a.
+// Split-KV MLA decode kernel for sm_100a, for s_q * h_q > 32 query rows.
 //
 // What it computes: for each chunk (request, range of 64-token blocks) that the
 // tile scheduler gave to this partition, the attention of one 128-row tile of
@@ -10,26 +10,39 @@
 //
 // B200 design (the pages' Hopper seesaw split of O over two warpgroups is
 // prior art; here the accumulators live in TMEM):
-//  * A CTA pair (cluster of 2) owns one 128-row tile.  A 128 x 512 fp32 output
-//    would fill all 512 TMEM columns of an SM, so CTA c keeps only its half
-//    O[:, 256c : 256c+256] (256 columns) and computes PV for that half.
-//  * The 576-deep Q.K^T contraction is split between the pair, so no MMA work
-//    is duplicated: CTA c contracts columns 256c .. 256c+255 plus its half of
-//    the 64 columns 512..575 (32 columns each).  The fp32 partial scores of a
-//    64-key block go to the peer through distributed shared memory (st.async
-//    completing on the peer's mbarrier); both CTAs then hold the same full
-//    scores and run the same softmax, so their two O halves stay consistent.
-//  * Each CTA TMA-loads 5 column boxes (64 cols = 128 B, 128-byte swizzle) of
-//    Q and of every page: boxes at columns 256c + {0,64,128,192} and 512.  The
-//    first four are also this CTA's V half (V = first 512 columns of K).
-//  * Warp roles: warp 0 lane 0 = TMA producer; warp 1 = TMEM owner, lane 0
-//    issues every tcgen05.mma; warps 4-7 = softmax / O correction / epilogue,
-//    one thread per query row (TMEM lane quadrant = warp % 4).
-//  * S = Q.K^T (M=128, N=64, K=16 x 18 steps, both operands K-major in smem);
-//    O += P.V (M=128, N=256, K=16 x 4 steps, P from TMEM, V MN-major in smem).
-//  * exp2 with log2(e) folded into the scale ("FlashMLA: 高性能GPU注意力机制计算库",
-//    4. Softmax数值稳定性优化).
-//  * EVICT_FIRST L2 policy on the page loads (细粒度流水线与缓存优化).
+//  * A 128 x 512 fp32 output tile alone fills the 512 TMEM columns of an SM, so
+//    a CTA pair (cluster of 2) owns one 128-row tile: CTA c keeps O[:, 256c :
+//    256c+256] and computes PV for that half.
+//  * The 576-deep Q.K^T contraction is split too, so no MMA work is
+//    duplicated: CTA c contracts columns 256c .. 256c+255 (its V half) plus the
+//    32 columns 512 + 32c ..  Those 256 main columns of Q stay in TMEM for the
+//    whole chunk (A operand from TMEM); the 32 others come from a
+//    shared-memory box.
+//  * The partial scores of a 64-key block are exchanged between the pair
+//    through distributed shared memory: rounded to 24 bits (sign, exponent, 15
+//    mantissa bits), staged, and moved by one bulk copy per warp that completes
+//    on the peer's mbarrier.  Both CTAs round both partials the same way, so
+//    they hold bit-identical scores and run the same softmax; their two O
+//    halves stay consistent.
+//  * The exchange runs one block ahead: right after combining block t, each
+//    softmax warp sends its partial of block t+1, which travels while block t's
+//    probabilities are computed.  A warp signals "slot consumed" with a relaxed
+//    arrive whose input depends on every word it read (a cluster-scope release
+//    there cost ~1000 cycles per block).
+//  * Each CTA TMA-loads, per page, four 64-column boxes (128-byte swizzle) at
+//    columns 256c + 64i -- also this CTA's V half -- and one 32-column box
+//    (64-byte swizzle) at 512 + 32c: 36 KB per page, four page stages, so the
+//    HBM latency of a page load hides behind three blocks of work; EVICT_FIRST
+//    L2 policy on page loads (细粒度流水线与缓存优化).
+//  * P goes to shared memory (K-major A operand of PV; V is the MN-major B
+//    operand read straight from the page tile).
+//  * Roles: warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0 issues every
+//    tcgen05.mma (Q.K^T two blocks ahead of P.V); warps 4-11 two per TMEM lane
+//    quadrant, one thread per (query row, half of the block's 64 keys): Q into
+//    TMEM, score exchange, softmax (exp2 with log2(e) folded into the scale,
+//    "FlashMLA: 高性能GPU注意力机制计算库" 4. Softmax数值稳定性优化), O correction,
+//    epilogue.  The two threads of a row agree on its maximum through shared
+//    memory and keep separate partial row sums, added at the end of a chunk.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -44,50 +57,58 @@ namespace splitkv {
 
 using namespace ptx;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kBlockN = kPage;              // keys per pipeline step
-constexpr int kBoxes = 5;                   // column boxes per CTA
-constexpr int kQBox = kTileRows * 128;      // 16 KB
-constexpr int kKBox = kBlockN * 128;        // 8 KB
-constexpr int kQBytes = kBoxes * kQBox;     // 80 KB
-constexpr int kStageBytes = kBoxes * kKBox; // 40 KB
-constexpr int kStages = 2;
-constexpr int kXWarp = 32 * kBlockN * 4;    // 8 KB: 32 rows x 64 fp32 partial scores
-constexpr int kXBytes = 4 * kXWarp;
-constexpr int kQkSteps = 18;                // 288 contraction columns / 16
+constexpr int kQrBox = kTileRows * 64;     // 8 KB: 128 rows x 32 columns (64-byte swizzle)
+constexpr int kKBox = kBlockN * 128;        // 8 KB: 64 keys x 64 columns (128-byte swizzle)
+constexpr int kKrBox = kBlockN * 64;        // 4 KB: 64 keys x 32 columns (64-byte swizzle)
+constexpr int kStageBytes = 4 * kKBox + kKrBox;  // 36 KB
+constexpr int kStages = 4;
+constexpr int kPBytes = kTileRows * 128;    // 16 KB: P, 128 rows x 64 keys (16-bit)
+constexpr int kSmWarps = 8;                 // softmax warps: 4 lane quadrants x 2 key halves
+constexpr int kHalfN = kBlockN / 2;         // keys per softmax thread
+constexpr int kRowWords = kHalfN * 3 / 4;   // 24 words: 32 scores at 24 bits
+constexpr int kRowBytes = kRowWords * 4;    // 96
+constexpr int kXWarp = 32 * kRowBytes;      // 3 KB per warp and direction
+constexpr int kXBytes = kSmWarps * kXWarp;  // 24 KB
 
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffX = kOffK + kStages * kStageBytes;
-constexpr int kOffBar = kOffX + kXBytes;
+constexpr int kOffQR = 0;                               // this CTA's 32 of Q's columns 512..575
+constexpr int kOffK = kOffQR + kQrBox;                  // page stages
+constexpr int kOffP = kOffK + kStages * kStageBytes;    // P
+constexpr int kOffStg = kOffP + kPBytes;                // send staging [8 warps]
+constexpr int kOffRcv = kOffStg + kXBytes;              // receive [8 warps]
+constexpr int kOffRed = kOffRcv + kXBytes;              // row maxima / sums [2 halves][128 rows]
+static_assert(kOffK % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "swizzle atom alignment");
+constexpr int kOffBar = kOffRed + 2 * kTileRows * 4;
 
 enum Bar {
   kKvFull = 0,
   kKvEmpty = kKvFull + kStages,
-  kQFull = kKvEmpty + kStages,
-  kQEmpty,
-  kSFull,
-  kSEmpty = kSFull + 2,
-  kPFull = kSEmpty + 2,
-  kPEmpty = kPFull + 2,
-  kODone = kPEmpty + 2,  // one phase per PV: the O correction waits for the previous PV
-  kOFinal,               // one phase per chunk: the epilogue waits for the chunk's last PV
-  kOEmpty,
-  kXFull,
-  kXEmpty = kXFull + 4,
-  kDrain = kXEmpty + 4,  // MMA thread: all of its tcgen05 ops have completed
+  kQrFull = kKvEmpty + kStages,  // Q column box 512..575 landed (TMA), one phase per chunk
+  kQtFull,                       // Q main columns written to TMEM (8 warps), one phase per chunk
+  kQEmpty,                       // the chunk's last Q.K^T completed
+  kSFull,                        // [2]
+  kSEmpty = kSFull + 2,          // [2], 8 warps
+  kPFull = kSEmpty + 2,          // 8 warps, one phase per block
+  kPEmpty,                       // one phase per P.V
+  kOFinal,                       // one phase per chunk: its last P.V completed
+  kOEmpty,                       // 8 warps, one phase per chunk
+  kXFull,                        // [8 warps]: the peer's partial landed
+  kXEmpty = kXFull + kSmWarps,   // [8 warps]: the peer consumed what this CTA sent
+  kRowX = kXEmpty + kSmWarps,    // [4 quadrants]: the two warps of a quadrant swap row values
+  kDrain = kRowX + 4,
   kNumBars
 };
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemUsed = kOffMisc + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0;    // 256 columns
-constexpr uint32_t kColS = 256;  // 2 x 64 columns
-constexpr uint32_t kColP = 384;  // 2 x 32 columns (16-bit pairs)
-
-__device__ __forceinline__ int box_col(int i, int crank) { return i < 4 ? 256 * crank + 64 * i : 512; }
+constexpr uint32_t kColO = 0;    // 256 columns: this CTA's half of O
+constexpr uint32_t kColS = 256;  // 2 x 64 columns: partial scores
+constexpr uint32_t kColQ = 384;  // 128 columns: Q columns 256c .. 256c+255 (16-bit pairs)
+static_assert(kColQ + 128 == kTmemCols, "TMEM budget");
 
 // The running maximum used as the exponent reference moves only when a new
 // score exceeds it by more than 2^8 (log2 units): the exponentials then stay
@@ -95,8 +116,6 @@ __device__ __forceinline__ int box_col(int i, int crank) { return i < 4 ? 256 * 
 // rescaled far less often, and the final out = O / l is unchanged because both
 // always share the same reference.
 constexpr float kRescaleThreshold = 8.0f;
-
-
 
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -109,9 +128,55 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   }
 }
 
+// The value a 24-bit packed score stands for (pack24 keeps the top three bytes;
+// unpack24 puts back a half step): the same bits without unpacking.
+__device__ __forceinline__ float round24(uint32_t v) { return __uint_as_float((v & 0xFFFFFF00u) | 0x80u); }
+
+// Walks a partition's blocks in order: chunk after chunk (one chunk = the
+// partition's blocks of one request), block after block.
+struct Walk {
+  int br, bk, er, ek;     // the partition's range from the scheduler
+  int req, blk, lo, hi, n;
+  int L;                  // cached tokens of the request
+  int chunk;              // chunk index within the partition
+  bool valid;
+
+  __device__ __forceinline__ void seek(const DecodeParams& p, int from) {
+    for (int r = from; r < p.batch && (r < er || (r == er && ek > 0)); ++r) {
+      L = p.cache_seqlens[r];
+      n = (L + kPage - 1) / kPage;
+      lo = (r == br) ? bk : 0;
+      hi = (r == er) ? ek : n;
+      if (hi > lo) {
+        req = r;
+        blk = lo;
+        valid = true;
+        return;
+      }
+    }
+    valid = false;
+  }
+  __device__ __forceinline__ void init(const DecodeParams& p, const int* meta) {
+    br = meta[0];
+    bk = meta[1];
+    er = meta[2];
+    ek = meta[3];
+    chunk = 0;
+    seek(p, br);
+  }
+  __device__ __forceinline__ void next(const DecodeParams& p) {
+    if (++blk < hi) return;
+    ++chunk;
+    seek(p, req + 1);
+  }
+  __device__ __forceinline__ bool first() const { return blk == lo; }
+  __device__ __forceinline__ bool last() const { return blk == hi - 1; }
+};
+
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    splitkv_pair_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+    splitkv_pair_kernel(const void* __restrict__ qptr, const __grid_constant__ CUtensorMap qrmap,
+                        const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap krmap,
                         const DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -127,16 +192,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = blockIdx.x >> 1;
   const int part = pair / p.m_tiles;
   const int mtile = pair % p.m_tiles;
-  const int* meta = p.meta + part * kMetaInts;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      uint32_t cnt = 1;
-      if (i == kSEmpty || i == kSEmpty + 1 || i == kPFull || i == kPFull + 1 || i == kOEmpty) cnt = 4;
-      mbar_init(bar(i), cnt);
+      const bool eight = i == kQtFull || i == kSEmpty || i == kSEmpty + 1 || i == kPFull || i == kOEmpty;
+      const bool two = i >= kRowX && i < kRowX + 4;
+      mbar_init(bar(i), eight ? static_cast<uint32_t>(kSmWarps) : two ? 2u : 1u);
     }
     *abort_flag = 0;
-    for (int w = 0; w < 4; ++w) mbar_arrive_expect_tx(bar(kXFull + w), kXWarp);  // arm phase 0
+    for (int i = 0; i < kSmWarps; ++i) mbar_arrive_expect_tx(bar(kXFull + i), kXWarp);  // arm phase 0
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -144,8 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (threadIdx.x == 32 * 2) {
-    prefetch_tmap(&qmap);
+    prefetch_tmap(&qrmap);
     prefetch_tmap(&kmap);
+    prefetch_tmap(&krmap);
   }
   tc_fence_before();
   __syncthreads();
@@ -157,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait_primary();
   if (threadIdx.x == 0) pdl_launch_dependents();
 
-  const int br = meta[0], bk = meta[1], er = meta[2], ek = meta[3], bs = meta[4];
+  const int* meta = p.meta + part * kMetaInts;
   const int R = p.rows;
   int* err = p.err;
 
@@ -165,36 +230,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t evict_first = policy_evict_first();
-      uint32_t it = 0, chunk = 0;
-      for (int req = br; req < p.batch && (req < er || (req == er && ek > 0)); ++req) {
-        const int L = p.cache_seqlens[req];
-        const int n = (L + kPage - 1) / kPage;
-        const int lo = (req == br) ? bk : 0;
-        const int hi = (req == er) ? ek : n;
-        if (hi <= lo) continue;
-        mbar_wait(bar(kQEmpty), (chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        mbar_arrive_expect_tx(bar(kQFull), kQBytes);
-        const int row0 = req * R + mtile * kTileRows;
-        for (int i = 0; i < kBoxes; ++i)
-          tma_load_2d(sbase + kOffQ + i * kQBox, &qmap, bar(kQFull), box_col(i, crank), row0);
-        const int32_t* bt = p.block_table + static_cast<int64_t>(req) * p.block_table_stride;
-        for (int blk = lo; blk < hi; ++blk, ++it) {
-          if (*abort_flag) break;
-          const int st = it % kStages;
-          mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-          int page = bt[blk];
-          if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
-            atomicOr(err, kDevErrPage);
-            atomicCAS(err + 1, 0, page == 0 ? -1 : page);
-            page = 0;
-          }
-          MLA_TR(kTrProd, it);
-          mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
-          for (int i = 0; i < kBoxes; ++i)
-            tma_load_3d_hint(sbase + kOffK + st * kStageBytes + i * kKBox, &kmap, bar(kKvFull + st),
-                             box_col(i, crank), 0, page, evict_first);
+      Walk w;
+      w.init(p, meta);
+      for (uint32_t it = 0; w.valid && !*abort_flag; ++it, w.next(p)) {
+        const int st = it % kStages;
+        mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        int page = p.block_table[static_cast<int64_t>(w.req) * p.block_table_stride + w.blk];
+        if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
+          atomicOr(err, kDevErrPage);
+          atomicCAS(err + 1, 0, page == 0 ? -1 : page);
+          page = 0;
         }
-        ++chunk;
+        mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
+        const uint32_t dst = sbase + kOffK + st * kStageBytes;
+        for (int i = 0; i < 4; ++i)  // columns 256c + 64i .. (also this CTA's V half)
+          tma_load_3d_hint(dst + i * kKBox, &kmap, bar(kKvFull + st), 256 * crank + 64 * i, 0, page, evict_first);
+        tma_load_3d_hint(dst + 4 * kKBox, &krmap, bar(kKvFull + st), 512 + 32 * crank, 0, page, evict_first);
+        if (w.first()) {
+          // the chunk's Q columns 512 + 32c .., once the previous chunk's last Q.K^T has read the old ones
+          mbar_wait(bar(kQEmpty), (w.chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          mbar_arrive_expect_tx(bar(kQrFull), kQrBox);
+          tma_load_2d(sbase + kOffQR, &qrmap, bar(kQrFull), 512 + 32 * crank, w.req * R + mtile * kTileRows);
+        }
       }
     }
   } else if (warp == 1) {
@@ -202,152 +259,301 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16(kBF16, kTileRows, kBlockN, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(kBF16, kTileRows, 256, false, true);
-      uint32_t it = 0, chunk = 0;
-      auto issue_pv = [&](uint32_t itp, int jjp, bool last) {
-        const int st = itp % kStages;
-        const int b = itp & 1;
-        if (jjp == 0) mbar_wait(bar(kOEmpty), (chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        mbar_wait(bar(kPFull + b), (itp >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      Walk wq, wp;
+      wq.init(p, meta);
+      wp = wq;
+      uint32_t tq = 0, tp = 0;
+      auto issue_qk = [&]() {
+        const int st = tq % kStages;
+        const int b = tq & 1;
+        if (wq.first()) {
+          mbar_wait(bar(kQrFull), wq.chunk & 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kQtFull), wq.chunk & 1, abort_flag, err, kDevErrTimeout);
+        }
+        mbar_wait(bar(kKvFull + st), (tq / kStages) & 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kSEmpty + b), ((tq >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         tc_fence_after();
-        MLA_TR(kTrPv, itp);
+        const uint32_t kbase = sbase + kOffK + st * kStageBytes;
+        const uint32_t dS = tmem + kColS + 64 * b;
+#pragma unroll
+        for (int s = 0; s < 16; ++s) {  // main columns: Q from TMEM
+          const uint64_t bdesc = smem_desc_sw128(kbase + (s >> 2) * kKBox + (s & 3) * 32, 16, 1024);
+          umma_ts(dS, tmem + kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {  // this CTA's 32 of the columns 512..575: Q from shared memory
+          const uint64_t adesc = smem_desc_sw64(sbase + kOffQR + i * 32, 16, 512);
+          const uint64_t bdesc = smem_desc_sw64(kbase + 4 * kKBox + i * 32, 16, 512);
+          umma_ss(dS, adesc, bdesc, idesc_qk, 1u);
+        }
+        umma_commit(bar(kSFull + b));
+        if (wq.last()) umma_commit(bar(kQEmpty));
+        wq.next(p);
+        ++tq;
+      };
+      auto issue_pv = [&]() {
+        const int st = tp % kStages;
+        if (wp.first()) mbar_wait(bar(kOEmpty), (wp.chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kPFull), tp & 1, abort_flag, err, kDevErrTimeout);
+        tc_fence_after();
         const uint32_t vbase = sbase + kOffK + st * kStageBytes;
+#pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          // V rows 16kk..16kk+15: 8-key groups 1024 B apart, 64-column boxes 8 KB apart
+          // P columns 16kk.. (K-major, 128 rows); V rows 16kk.. (MN-major: 64-column boxes 8 KB apart)
+          const uint64_t adesc = smem_desc_sw128(sbase + kOffP + kk * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, kKBox, 1024);
-          umma_ts(tmem + kColO, tmem + kColP + 32 * b + 8 * kk, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
+          umma_ss(tmem + kColO, adesc, bdesc, idesc_pv, (!wp.first() || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar(kKvEmpty + st));
-        umma_commit(bar(kPEmpty + b));
-        umma_commit(bar(kODone));
-        if (last) umma_commit(bar(kOFinal));
+        umma_commit(bar(kPEmpty));
+        if (wp.last()) umma_commit(bar(kOFinal));
+        wp.next(p);
+        ++tp;
       };
-      for (int req = br; req < p.batch && (req < er || (req == er && ek > 0)); ++req) {
-        const int L = p.cache_seqlens[req];
-        const int n = (L + kPage - 1) / kPage;
-        const int lo = (req == br) ? bk : 0;
-        const int hi = (req == er) ? ek : n;
-        if (hi <= lo) continue;
-        const int nb = hi - lo;
-        mbar_wait(bar(kQFull), chunk & 1, abort_flag, err, kDevErrTimeout);
-        tc_fence_after();
-        if (*abort_flag) break;
-        for (int jj = 0; jj < nb; ++jj) {
-          const uint32_t itc = it + jj;
-          const int st = itc % kStages;
-          const int b = itc & 1;
-          mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, abort_flag, err, kDevErrTimeout);
-          mbar_wait(bar(kSEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-          tc_fence_after();
-          MLA_TR(kTrQk, itc);
-          const uint32_t kbase = sbase + kOffK + st * kStageBytes;
-          for (int s = 0; s < kQkSteps; ++s) {
-            const int box = s < 16 ? s / 4 : 4;
-            const int kk = s < 16 ? s % 4 : 2 * static_cast<int>(crank) + (s - 16);
-            const uint64_t adesc = smem_desc_sw128(sbase + kOffQ + box * kQBox + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(kbase + box * kKBox + kk * 32, 16, 1024);
-            umma_ss(tmem + kColS + 64 * b, adesc, bdesc, idesc_qk, s > 0 ? 1u : 0u);
-          }
-          umma_commit(bar(kSFull + b));
-          if (jj == nb - 1) umma_commit(bar(kQEmpty));
-          if (jj > 0) issue_pv(itc - 1, jj - 1, false);
-        }
-        issue_pv(it + nb - 1, nb - 1, true);
-        it += nb;
-        ++chunk;
+      // Q.K^T runs two blocks ahead of P.V: the softmax warps release a score
+      // buffer as soon as they have combined it with the peer's partial.
+      for (int i = 0; i < 2 && wq.valid; ++i) issue_qk();
+      while (wp.valid && !*abort_flag) {
+        if (wq.valid) issue_qk();
+        issue_pv();
       }
       umma_commit(bar(kDrain));
       mbar_wait_drain(bar(kDrain), 0);
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax / correction / epilogue
+    // ------------------------------------------------------------ Q to TMEM, exchange, softmax, correction, epilogue
+    // Two warps per TMEM lane quadrant: warp 4 + q4 takes keys 0..31 of its 32 rows, warp 8 + q4
+    // keys 32..63; both keep the same row maximum (shared through shared memory).
+    const int sm = warp - 4;          // 0..7
     const int q4 = warp & 3;
+    const int half = sm >> 2;
     const int row = q4 * 32 + lane;
     const int row_g = mtile * kTileRows + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    float* xrow = reinterpret_cast<float*>(smem + kOffX + q4 * kXWarp + lane * (kBlockN * 4));
-    const uint32_t xrow_remote = mapa(smem_u32(xrow), peer);
-    const uint32_t xfull_remote = mapa(bar(kXFull + q4), peer);
-    const uint32_t xempty_remote = mapa(bar(kXEmpty + q4), peer);
-    const int sw = lane & 15;
-    // a warp whose 32 rows are all padding (rows >= s_q * h_q) keeps the
-    // barrier protocol but skips the math; its peer warp skips the same way
+    uint8_t* stg_row = smem + kOffStg + sm * kXWarp + lane * kRowBytes;
+    const uint32_t stg_warp = sbase + kOffStg + sm * kXWarp;
+    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [half][row]
+    uint32_t rx_phase = 0;
+    // the other half's value of this row (both halves call it with their own); two phases of the
+    // quadrant's barrier: values written, then values read (before either half writes again)
+    auto row_swap = [&](float v) {
+      red[half * kTileRows + row] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kRowX + q4));
+      mbar_wait(bar(kRowX + q4), rx_phase & 1, abort_flag, err, kDevErrTimeout);
+      const float o = red[(half ^ 1) * kTileRows + row];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kRowX + q4));
+      mbar_wait(bar(kRowX + q4), (rx_phase + 1) & 1, abort_flag, err, kDevErrTimeout);
+      rx_phase += 2;
+      return o;
+    };
+    // 16-byte chunk order within a 96-byte row: lanes i and i+4 of each group of 8 differ
+    const int sw = (lane >> 2) & 1;
+    // a quadrant whose 32 rows are all padding keeps the barrier protocol but skips the math;
+    // its peer quadrant skips the same way
     const bool active = mtile * kTileRows + q4 * 32 < R;
-    uint32_t it = 0, chunk = 0;
-    for (int req = br; req < p.batch && (req < er || (req == er && ek > 0)); ++req) {
-      const int L = p.cache_seqlens[req];
-      const int n = (L + kPage - 1) / kPage;
-      const int lo = (req == br) ? bk : 0;
-      const int hi = (req == er) ? ek : n;
-      if (hi <= lo) continue;
-      const int nb = hi - lo;
-      int limit = 0;
-      if (row_g < R) {
-        limit = p.causal ? L - (p.s_q - 1 - row_g / p.h_q) : L;
-        limit = limit < 0 ? 0 : limit;
-      }
-      float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: row sum relative to it
-      for (int jj = 0; jj < nb; ++jj) {
-        const uint32_t itc = it + jj;
-        const int b = itc & 1;
-        float x[64];
-        mbar_wait(bar(kSFull + b), (itc >> 1) & 1, abort_flag, err, kDevErrTimeout);
-        __syncwarp();  // reconverge before the warp-collective tcgen05.ld
-        tc_fence_after();
-        if (lane == 0) MLA_TR(kTrSmS, itc);
-        if (active) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(t_lane + kColS + 64 * b, r0);
-          tmem_ld32(t_lane + kColS + 64 * b + 32, r1);
-          tmem_wait_ld();
+#ifdef MLA_TRACE
+    // developer builds: cycles spent per section, summed over the blocks
+    long long tr_acc[kTrNum] = {};
+    long long tr_prev = clock64();
+#endif
+    auto stamp = [&](int ev, uint32_t) {
+#ifdef MLA_TRACE
+      const long long now = clock64();
+      tr_acc[ev] += now - tr_prev;
+      tr_prev = now;
+#endif
+      (void)ev;
+    };
+
+    // Q columns 256c + 128h .. +127 of this thread's row of request `req` -> TMEM columns kColQ + 64h ..
+    auto q_row = [&](int req) {
+      return reinterpret_cast<const uint8_t*>(qptr) +
+             ((static_cast<int64_t>(req) * R + (row_g < R ? row_g : 0)) * kDK + 256 * crank + 128 * half) * 2;
+    };
+    auto prefetch_q = [&](int req) {
+      if (row_g >= R) return;
+      const uint8_t* q = q_row(req);
+      prefetch_l1(q);
+      prefetch_l1(q + 128);
+    };
+    auto store_q = [&](int req) {
+      const uint4* qrow = reinterpret_cast<const uint4*>(q_row(req));
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            x[c] = __uint_as_float(r0[c]);
-            x[32 + c] = __uint_as_float(r1[c]);
-          }
+      for (int c32 = 0; c32 < 2; ++c32) {
+        uint32_t w[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 d = make_uint4(0, 0, 0, 0);
+          if (row_g < R) d = __ldg(qrow + c32 * 8 + v);
+          w[4 * v] = d.x;
+          w[4 * v + 1] = d.y;
+          w[4 * v + 2] = d.z;
+          w[4 * v + 3] = d.w;
         }
+        tmem_st32(t_lane + kColQ + 64 * half + 32 * c32, w);
+      }
+      tmem_wait_st();
+    };
+
+    // Block u's scores are ready: (if u ends its chunk and another chunk follows) put the next
+    // chunk's Q into TMEM, then send this warp's part of the partial scores to the peer.
+    auto send_partial = [&](uint32_t u, const Walk& wu) {
+      const int b = u & 1;
+      Walk nx = wu;
+      nx.next(p);
+      const bool new_q = nx.valid && nx.chunk != wu.chunk;
+      if (new_q && active) prefetch_q(nx.req);  // into L1 while the scores finish
+      mbar_wait(bar(kSFull + b), (u >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      __syncwarp();  // reconverge before the warp-collective tcgen05 ops
+      tc_fence_after();
+      if (new_q) {
+        // the Q.K^T of block u was the chunk's last: the Q columns are free
+        mbar_wait(bar(kQEmpty), wu.chunk & 1, abort_flag, err, kDevErrTimeout);
+        __syncwarp();
+        tc_fence_after();
+        if (active) store_q(nx.req);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kSEmpty + b));
-        if (!active) {
-          mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kPFull + b));
-          continue;
-        }
+        if (lane == 0) mbar_arrive(bar(kQtFull));
+      }
+      stamp(kTrSmS, u);
+      if (!active) return;
+      uint32_t r[32];
+      tmem_ld32(t_lane + kColS + 64 * b + kHalfN * half, r);
+      tmem_wait_ld();
+      stamp(kTrA, u);
+      if (lane == 0) bulk_wait_read_all();  // the previous copy out of the staging row is done
+      __syncwarp();
+      stamp(kTrB, u);
+#pragma unroll
+      for (int k = 0; k < kRowWords / 12; ++k) {  // 16 scores -> 12 words -> 3 chunks
+        uint32_t w[12];
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          pack24(r[16 * k + 4 * g], r[16 * k + 4 * g + 1], r[16 * k + 4 * g + 2], r[16 * k + 4 * g + 3], w[3 * g],
+                 w[3 * g + 1], w[3 * g + 2]);
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+          *reinterpret_cast<uint4*>(stg_row + (((3 * k + j) ^ sw) << 4)) =
+              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+      }
+      fence_proxy_async_smem();  // the bulk copy reads the staging through the async proxy
+      __syncwarp();
+      stamp(kTrC, u);
+      if (lane == 0) {
+        // the peer's receive slot of this warp is free once the peer has combined block u - 1
+        mbar_wait<true>(bar(kXEmpty + sm), (u & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        bulk_copy_to_peer(mapa(sbase + kOffRcv + sm * kXWarp, peer), stg_warp, kXWarp, mapa(bar(kXFull + sm), peer));
+        bulk_commit_group();
+      }
+      __syncwarp();
+      stamp(kTrSend, u);
+    };
 
-        // exchange partial scores with the peer CTA (same rows, other half of the contraction)
-        mbar_wait<true>(bar(kXEmpty + q4), (itc & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+    Walk wu, wt;
+    wu.init(p, meta);
+    wt = wu;
+    if (wu.valid) {  // the first chunk's Q, and the first block's partial
+      if (active) store_q(wu.req);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kQtFull));
+      send_partial(0, wu);
+      wu.next(p);
+    }
+    uint32_t u = 1;
+    float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: this half's row sum relative to it
+    for (uint32_t t = 0; wt.valid; ++t, wt.next(p)) {
+      if (*abort_flag) break;
+      // ---- block t: own partial (rounded as sent) + the peer's, then release the score buffer
+      const int b = t & 1;
+      float x[kHalfN];
+      if (active) {
+        mbar_wait<true>(bar(kXFull + sm), t & 1, abort_flag, err, kDevErrTimeout);
+        __syncwarp();
+        stamp(kTrSmX, t);
+        uint32_t r[32];
+        tmem_ld32(t_lane + kColS + 64 * b + kHalfN * half, r);
+        tmem_wait_ld();
+        stamp(kTrD, t);
+        const uint8_t* rcv_row = smem + kOffRcv + sm * kXWarp + lane * kRowBytes;
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const int pos = c4 ^ sw;
-          st_async_v4(xrow_remote + pos * 16, xfull_remote, x[4 * c4], x[4 * c4 + 1], x[4 * c4 + 2], x[4 * c4 + 3]);
-        }
-        mbar_wait<true>(bar(kXFull + q4), itc & 1, abort_flag, err, kDevErrTimeout);
+        for (int k = 0; k < kRowWords / 12; ++k) {  // 3 chunks = 16 scores per step
+          const uint4 c0 = *reinterpret_cast<const uint4*>(rcv_row + (((3 * k) ^ sw) << 4));
+          const uint4 c1 = *reinterpret_cast<const uint4*>(rcv_row + (((3 * k + 1) ^ sw) << 4));
+          const uint4 c2 = *reinterpret_cast<const uint4*>(rcv_row + (((3 * k + 2) ^ sw) << 4));
+          const uint32_t wv[12] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const int pos = c4 ^ sw;
-          const float4 y = *reinterpret_cast<const float4*>(xrow + pos * 4);
-          x[4 * c4] += y.x;
-          x[4 * c4 + 1] += y.y;
-          x[4 * c4 + 2] += y.z;
-          x[4 * c4 + 3] += y.w;
+          for (int g = 0; g < 4; ++g) {
+            float a0, a1, a2, a3;
+            unpack24(wv[3 * g], wv[3 * g + 1], wv[3 * g + 2], a0, a1, a2, a3);
+            const int c = 16 * k + 4 * g;
+            x[c] = round24(r[c]) + a0;
+            x[c + 1] = round24(r[c + 1]) + a1;
+            x[c + 2] = round24(r[c + 2]) + a2;
+            x[c + 3] = round24(r[c + 3]) + a3;
+          }
         }
+        stamp(kTrE, t);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kSEmpty + b));  // Q.K^T of block t + 2 may overwrite the scores
+      stamp(kTrSmC, t);
+
+      if (wt.first()) {
+        m = -INFINITY;
+        l = 0.f;
+      }
+      float mx = -INFINITY;  // this half's maximum of the block's scaled scores
+      if (active) {
+        // ---- online softmax in log2 units
+        int limit = 0;
+        if (row_g < R) {
+          limit = p.causal ? wt.L - (p.s_q - 1 - row_g / p.h_q) : wt.L;
+          limit = limit < 0 ? 0 : limit;
+        }
+        const int kbase = wt.blk * kBlockN + kHalfN * half;
+        if (__all_sync(0xffffffffu, kbase + kHalfN <= limit)) {
+#pragma unroll
+          for (int c = 0; c < kHalfN; ++c) {
+            x[c] *= p.scale_log2;
+            mx = fmaxf(mx, x[c]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kHalfN; ++c) {
+            x[c] = (kbase + c < limit) ? x[c] * p.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, x[c]);
+          }
+        }
+        stamp(kTrF, t);
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar(kXFull + q4), kXWarp);  // arm the next phase first
-          mbar_arrive_cluster(xempty_remote);               // then let the peer send again
-          MLA_TR(kTrSmX, itc);
+          // every lane's mx was computed from every word it read from the receive slot, so those
+          // reads are complete: arm the slot's next phase, then let the peer refill it (a relaxed
+          // arrive; a release at cluster scope costs ~1000 cycles here)
+          mbar_arrive_expect_tx(bar(kXFull + sm), kXWarp);
+          mbar_arrive_cluster_relaxed_after(mapa(bar(kXEmpty + sm), peer), mx);
         }
-
-        // online softmax in log2 units
-        const int kbase = (lo + jj) * kBlockN;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float t = (kbase + c < limit) ? x[c] * p.scale_log2 : -INFINITY;
-          x[c] = t;
-          mx = fmaxf(mx, t);
-        }
+        __syncwarp();
+        stamp(kTrQk, t);
+      }
+      if (wu.valid) {  // block t + 1's partial travels while block t's softmax runs
+        send_partial(u, wu);
+        wu.next(p);
+        ++u;
+      }
+      if (!active) {
+        mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kPFull));
+      } else {
+        // both halves of the row take the same maximum
+        mx = fmaxf(mx, row_swap(mx));
+        stamp(kTrG, t);
         bool resc = false;
         float alpha = 1.f;
         if (mx > m + kRescaleThreshold) {  // also true when m is still -inf and a key is visible
@@ -358,65 +564,80 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = mx;
         }
         const float base = (m == -INFINITY) ? 0.f : m;
-        float sum = 0.f;
-        uint32_t pk[32];
+        float s0 = 0.f, s1 = 0.f;
+        uint32_t pk[kHalfN / 2];
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
+        for (int c2 = 0; c2 < kHalfN / 2; ++c2) {
           const float p0 = ex2(x[2 * c2] - base);
           const float p1 = ex2(x[2 * c2 + 1] - base);
-          sum += p0 + p1;
+          s0 += p0;
+          s1 += p1;
           pk[c2] = pack2<kBF16>(p0, p1);
         }
-        l = l * alpha + sum;
+        l = l * alpha + (s0 + s1);
+        stamp(kTrH, t);
 
-        mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        // P (this half's 32 keys of the row), once the previous P.V has read P (so O also holds
+        // every earlier block)
+        mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
         tc_fence_after();
-        tmem_st32(t_lane + kColP + 32 * b, pk);
-        if (__any_sync(0xffffffffu, resc && jj > 0)) {
-          // O holds PV of blocks before this one (jj == 0 is overwritten by its own PV)
-          mbar_wait(bar(kODone), (itc - 1) & 1, abort_flag, err, kDevErrTimeout);
-          __syncwarp();
-          tc_fence_after();
+        {
+          uint8_t* prow = smem + kOffP + row * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint4*>(prow + (((4 * half + k) ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+        }
+        fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+        if (__any_sync(0xffffffffu, resc)) {
+          // only blocks after the chunk's first can move an established reference, so O holds
+          // the chunk's earlier blocks here; each half rescales 128 of the 256 columns
 #pragma unroll 1
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 4; ++k) {
             uint32_t o[32];
-            tmem_ld32(t_lane + kColO + 32 * k, o);
+            const uint32_t ta = t_lane + kColO + 128 * half + 32 * k;
+            tmem_ld32(ta, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(t_lane + kColO + 32 * k, o);
+            tmem_st32(ta, o);
           }
+          tmem_wait_st();
         }
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          MLA_TR(kTrSmP, itc);
-          mbar_arrive(bar(kPFull + b));
-        }
+        if (lane == 0) mbar_arrive(bar(kPFull));
+        __syncwarp();
+        stamp(kTrSmP, t);
       }
 
-      // epilogue: normalise this CTA's O half and write it
-      mbar_wait(bar(kOFinal), chunk & 1, abort_flag, err, kDevErrTimeout);
+      if (!wt.last()) continue;
+      // ---- epilogue of the chunk: normalise this CTA's O half and write it
+      float lt = 0.f;
+      if (active) {
+        const float lo = row_swap(l);
+        lt = half == 0 ? l + lo : lo + l;  // same order in both halves
+      }
+      mbar_wait(bar(kOFinal), wt.chunk & 1, abort_flag, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
       if (active) {
-        const bool whole = (lo == 0 && hi == n);
-        const int split_idx = (req == br) ? bs : 0;
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const float lse_v = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        const int64_t chunk_row = whole ? 0 : (static_cast<int64_t>(p.num_splits[req] + split_idx) * R + row_g);
+        const bool whole = (wt.lo == 0 && wt.hi == wt.n);
+        const int split_idx = (wt.req == wt.br) ? meta[4] : 0;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const int64_t chunk_row =
+            whole ? 0 : (static_cast<int64_t>(p.num_splits[wt.req] + split_idx) * R + row_g);
 #pragma unroll 1
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
           uint32_t o[32];
-          tmem_ld32(t_lane + kColO + 32 * k, o);
+          tmem_ld32(t_lane + kColO + 128 * half + 32 * k, o);
           tmem_wait_ld();
           if (row_g < R) {
-            const int col = static_cast<int>(crank) * 256 + 32 * k;
+            const int col = static_cast<int>(crank) * 256 + 128 * half + 32 * k;
             if (whole) {
               uint4* dst = reinterpret_cast<uint4*>(
-                  reinterpret_cast<uint16_t*>(p.out) + (static_cast<int64_t>(req) * R + row_g) * kDV + col);
+                  reinterpret_cast<uint16_t*>(p.out) + (static_cast<int64_t>(wt.req) * R + row_g) * kDV + col);
 #pragma unroll
               for (int v = 0; v < 4; ++v) {
                 uint4 w;
@@ -435,10 +656,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (crank == 0 && row_g < R) {
+        if (crank == 0 && half == 0 && row_g < R) {
+          const float lse_v = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
           if (whole) {
             const int s = row_g / p.h_q, h = row_g % p.h_q;
-            p.lse[static_cast<int64_t>(req) * R + h * p.s_q + s] = lse_v;
+            p.lse[static_cast<int64_t>(wt.req) * R + h * p.s_q + s] = lse_v;
           } else {
             p.lse_acc[chunk_row] = lse_v;
           }
@@ -447,9 +669,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kOEmpty));
-      it += nb;
-      ++chunk;
+      stamp(kTrProd, t);  // epilogue
     }
+    if (lane == 0) bulk_wait_read_all();
+#ifdef MLA_TRACE
+    if (lane == 0 && p.trace && blockIdx.x < 2)
+      for (int e = 0; e < kTrNum; ++e) p.trace[(blockIdx.x * kTrNum + e) * kTrMax + sm] = tr_acc[e];
+#endif
   }
 
   // ------------------------------------------------------------ teardown
@@ -466,14 +692,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace splitkv
 
 int splitkv_smem_bytes() { return splitkv::kSmemBytes; }
+int splitkv_threads() { return splitkv::kThreads; }
 
 const void* splitkv_kernel_ptr(bool bf16) {
   return bf16 ? reinterpret_cast<const void*>(&splitkv::splitkv_pair_kernel<true>)
               : reinterpret_cast<const void*>(&splitkv::splitkv_pair_kernel<false>);
 }
 
-cudaError_t launch_splitkv(bool bf16, const CUtensorMap& qmap, const CUtensorMap& kmap, const DecodeParams& p,
-                           cudaStream_t stream) {
+cudaError_t launch_splitkv(bool bf16, const void* q, const CUtensorMap& qrmap, const CUtensorMap& kmap,
+                           const CUtensorMap& krmap, const DecodeParams& p, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * p.num_parts * p.m_tiles);  // one cluster of 2 CTAs per (partition, row tile)
   cfg.blockDim = dim3(splitkv::kThreads);
@@ -488,8 +715,8 @@ cudaError_t launch_splitkv(bool bf16, const CUtensorMap& qmap, const CUtensorMap
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (bf16) return cudaLaunchKernelEx(&cfg, splitkv::splitkv_pair_kernel<true>, qmap, kmap, p);
-  return cudaLaunchKernelEx(&cfg, splitkv::splitkv_pair_kernel<false>, qmap, kmap, p);
+  if (bf16) return cudaLaunchKernelEx(&cfg, splitkv::splitkv_pair_kernel<true>, q, qrmap, kmap, krmap, p);
+  return cudaLaunchKernelEx(&cfg, splitkv::splitkv_pair_kernel<false>, q, qrmap, kmap, krmap, p);
 }
 
 }  // namespace mla
