@@ -150,16 +150,23 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
-def profile_traffic(name: str):
-    """DRAM bytes per split-KV launch from the committed ncu summary, if it is for this source."""
-    path = os.path.join(ROOT, "profiles", f"splitkv_{name}.md")
-    src = os.path.join(ROOT, "mla_decode_attention_16_b200", "csrc", "splitkv.cu")
+def kernel_of(rows: int):
+    """(name, source file) of the split-KV kernel the library runs for s_q * h_q = rows."""
+    if rows <= 32:
+        return "splitkv_narrow_kernel", "splitkv_narrow.cu"
+    return "splitkv_pair_kernel", "splitkv.cu"
+
+
+def profile_traffic(name: str, kernel: str, source: str):
+    """DRAM bytes per split-KV launch from the committed ncu summary, if it was taken from this source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{name}.md")
+    src = os.path.join(ROOT, "mla_decode_attention_16_b200", "csrc", source)
     try:
         text = open(path).read()
         digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except OSError:
         return None
-    m_sha = re.search(r"splitkv\.cu sha256\[:16\]:\s*([0-9a-f]{16})", text)
+    m_sha = re.search(re.escape(source) + r" sha256\[:16\]:\s*([0-9a-f]{16})", text)
     m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if not m_sha or not m_tr or m_sha.group(1) != digest:
         return None
@@ -368,9 +375,10 @@ def run_gpu(args, name: str):
         achieved = cost["flops"] / kern_s / 1e12
         peak = float(peaks["bf16_tflops"])  # fp16 dense tensor rate equals bf16 on this part
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
-    roof["traffic"] = profile_traffic(name)
+    kname, ksrc = kernel_of(inp.s_q * inp.h_q)
+    roof["traffic"] = profile_traffic(name, kname, ksrc)
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["kernel"] = "splitkv_pair_kernel"
+    roof["kernel"] = kname
     roof["kernel_us"] = kern_s * 1e6
     roof["algorithmic_per_launch"] = cost["bytes"] if unit == "GB/s" else cost["flops"]
 
