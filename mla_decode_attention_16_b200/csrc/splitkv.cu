@@ -77,9 +77,9 @@ constexpr int kOffK = kOffQR + kQrBox;                  // page stages
 constexpr int kOffP = kOffK + kStages * kStageBytes;    // P
 constexpr int kOffStg = kOffP + kPBytes;                // send staging [8 warps]
 constexpr int kOffRcv = kOffStg + kXBytes;              // receive [8 warps]
-constexpr int kOffRed = kOffRcv + kXBytes;              // row maxima / sums [2 halves][128 rows]
+constexpr int kOffRed = kOffRcv + kXBytes;              // row maxima / sums [2 parities][2 halves][128 rows]
 static_assert(kOffK % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "swizzle atom alignment");
-constexpr int kOffBar = kOffRed + 2 * kTileRows * 4;
+constexpr int kOffBar = kOffRed + 2 * 2 * kTileRows * 4;
 
 enum Bar {
   kKvFull = 0,
@@ -173,6 +173,24 @@ struct Walk {
   __device__ __forceinline__ bool last() const { return blk == hi - 1; }
 };
 
+// Developer builds (MLA_TRACE): cycles a single-thread role spends in one kind of wait.
+struct WaitClock {
+#ifdef MLA_TRACE
+  long long acc[6] = {};
+  long long t0 = 0;
+  __device__ __forceinline__ void start() { t0 = clock64(); }
+  __device__ __forceinline__ void stop(int slot) { acc[slot] += clock64() - t0; }
+  __device__ __forceinline__ void dump(const DecodeParams& p, int column) const {
+    if (p.trace && blockIdx.x < 2)
+      for (int e = 0; e < 6; ++e) p.trace[(blockIdx.x * kTrNum + e) * kTrMax + column] = acc[e];
+  }
+#else
+  __device__ __forceinline__ void start() {}
+  __device__ __forceinline__ void stop(int) {}
+  __device__ __forceinline__ void dump(const DecodeParams&, int) const {}
+#endif
+};
+
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_pair_kernel(const void* __restrict__ qptr, const __grid_constant__ CUtensorMap qrmap,
@@ -232,10 +250,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t evict_first = policy_evict_first();
       Walk w;
       w.init(p, meta);
-      for (uint32_t it = 0; w.valid && !*abort_flag; ++it, w.next(p)) {
+      WaitClock wc;
+      auto page_of = [&](const Walk& x) {
+        return x.valid ? p.block_table[static_cast<int64_t>(x.req) * p.block_table_stride + x.blk] : 0;
+      };
+      int page_next = page_of(w);
+      for (uint32_t it = 0; w.valid && !*abort_flag; ++it) {
         const int st = it % kStages;
+        int page = page_next;
+        Walk nx = w;
+        nx.next(p);
+        page_next = page_of(nx);  // the next block's page index is read while this stage frees up
+        wc.start();
         mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        int page = p.block_table[static_cast<int64_t>(w.req) * p.block_table_stride + w.blk];
+        wc.stop(0);
         if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
           atomicOr(err, kDevErrPage);
           atomicCAS(err + 1, 0, page == 0 ? -1 : page);
@@ -248,11 +276,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_hint(dst + 4 * kKBox, &krmap, bar(kKvFull + st), 512 + 32 * crank, 0, page, evict_first);
         if (w.first()) {
           // the chunk's Q columns 512 + 32c .., once the previous chunk's last Q.K^T has read the old ones
+          wc.start();
           mbar_wait(bar(kQEmpty), (w.chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          wc.stop(1);
           mbar_arrive_expect_tx(bar(kQrFull), kQrBox);
           tma_load_2d(sbase + kOffQR, &qrmap, bar(kQrFull), 512 + 32 * crank, w.req * R + mtile * kTileRows);
         }
+        w = nx;
       }
+      wc.dump(p, 9);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -263,15 +295,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       wq.init(p, meta);
       wp = wq;
       uint32_t tq = 0, tp = 0;
+      WaitClock wc;
+      // Inputs of the next Q.K^T (chunk's Q, the page, a free score buffer) / the next P.V (P, and
+      // for a chunk's first block the epilogue having read O) are complete.  Each barrier phase
+      // tested here cannot run a full phase ahead: its producer waits on this thread's earlier work.
+      auto qk_ready = [&]() {
+        if (wq.first() && !(mbar_test_wait(bar(kQrFull), wq.chunk & 1) && mbar_test_wait(bar(kQtFull), wq.chunk & 1)))
+          return false;
+        return mbar_test_wait(bar(kKvFull + tq % kStages), (tq / kStages) & 1) &&
+               mbar_test_wait(bar(kSEmpty + (tq & 1)), ((tq >> 1) & 1) ^ 1);
+      };
+      auto pv_ready = [&]() {
+        if (wp.first() && !mbar_test_wait(bar(kOEmpty), (wp.chunk & 1) ^ 1)) return false;
+        return mbar_test_wait(bar(kPFull), tp & 1);
+      };
       auto issue_qk = [&]() {
         const int st = tq % kStages;
         const int b = tq & 1;
-        if (wq.first()) {
-          mbar_wait(bar(kQrFull), wq.chunk & 1, abort_flag, err, kDevErrTimeout);
-          mbar_wait(bar(kQtFull), wq.chunk & 1, abort_flag, err, kDevErrTimeout);
-        }
-        mbar_wait(bar(kKvFull + st), (tq / kStages) & 1, abort_flag, err, kDevErrTimeout);
-        mbar_wait(bar(kSEmpty + b), ((tq >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         tc_fence_after();
         const uint32_t kbase = sbase + kOffK + st * kStageBytes;
         const uint32_t dS = tmem + kColS + 64 * b;
@@ -293,8 +333,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto issue_pv = [&]() {
         const int st = tp % kStages;
-        if (wp.first()) mbar_wait(bar(kOEmpty), (wp.chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        mbar_wait(bar(kPFull), tp & 1, abort_flag, err, kDevErrTimeout);
         tc_fence_after();
         const uint32_t vbase = sbase + kOffK + st * kStageBytes;
 #pragma unroll
@@ -310,15 +348,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         wp.next(p);
         ++tp;
       };
-      // Q.K^T runs two blocks ahead of P.V: the softmax warps release a score
-      // buffer as soon as they have combined it with the peer's partial.
-      for (int i = 0; i < 2 && wq.valid; ++i) issue_qk();
-      while (wp.valid && !*abort_flag) {
-        if (wq.valid) issue_qk();
-        issue_pv();
+      // Whichever is ready first: a P.V frees its page stage, so it goes before a ready Q.K^T;
+      // Q.K^T may be issued up to three blocks ahead of P.V (the two score buffers bound it too).  A bounded wait covers the
+      // time nothing is ready.
+      long long idle_since = clock64();
+      uint32_t polls = 0;
+      while (wp.valid) {
+        if (tp < tq && pv_ready()) {
+          issue_pv();
+        } else if (wq.valid && tq < tp + 3 && qk_ready()) {
+          issue_qk();
+        } else {
+          if ((++polls & 15u) == 0) {
+            if (*abort_flag) break;
+            const long long now = clock64();
+            if (now - idle_since > kWaitCycles) {
+              *abort_flag = 1;
+              atomicOr(err, kDevErrTimeout);
+              break;
+            }
+          }
+          continue;
+        }
+        idle_since = clock64();
       }
       umma_commit(bar(kDrain));
       mbar_wait_drain(bar(kDrain), 0);
+      wc.dump(p, 8);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ Q to TMEM, exchange, softmax, correction, epilogue
@@ -332,20 +388,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     uint8_t* stg_row = smem + kOffStg + sm * kXWarp + lane * kRowBytes;
     const uint32_t stg_warp = sbase + kOffStg + sm * kXWarp;
-    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [half][row]
+    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [parity][half][row]
     uint32_t rx_phase = 0;
-    // the other half's value of this row (both halves call it with their own); two phases of the
-    // quadrant's barrier: values written, then values read (before either half writes again)
+    // the other half's value of this row (both halves call it with their own): one phase of the
+    // quadrant's barrier per swap; the two parities of the buffer keep a fast half's next write
+    // off the slot the other half may still be reading (it cannot write twice ahead: the swap
+    // after next waits for the other half's arrival of the next one)
     auto row_swap = [&](float v) {
-      red[half * kTileRows + row] = v;
+      float* slot = red + (rx_phase & 1) * 2 * kTileRows;
+      slot[half * kTileRows + row] = v;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kRowX + q4));
       mbar_wait(bar(kRowX + q4), rx_phase & 1, abort_flag, err, kDevErrTimeout);
-      const float o = red[(half ^ 1) * kTileRows + row];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kRowX + q4));
-      mbar_wait(bar(kRowX + q4), (rx_phase + 1) & 1, abort_flag, err, kDevErrTimeout);
-      rx_phase += 2;
+      const float o = slot[(half ^ 1) * kTileRows + row];
+      ++rx_phase;
       return o;
     };
     // 16-byte chunk order within a 96-byte row: lanes i and i+4 of each group of 8 differ

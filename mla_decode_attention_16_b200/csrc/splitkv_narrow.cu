@@ -196,11 +196,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       Chunk ch;
       while (!*abort_flag && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
         const int32_t* bt = p.block_table + static_cast<int64_t>(ch.req) * p.block_table_stride;
+        int page_next = bt[ch.lo];
         for (int blk = ch.lo; blk < ch.hi; ++blk, ++it) {
           if (*abort_flag) break;
           const int st = it % kStages;
+          int page = page_next;
+          if (blk + 1 < ch.hi) page_next = bt[blk + 1];  // read while this stage frees up
           mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-          int page = bt[blk];
           if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
             atomicOr(err, kDevErrPage);
             atomicCAS(err + 1, 0, page == 0 ? -1 : page);
