@@ -63,7 +63,24 @@ __device__ __forceinline__ void trace_stamp(const DecodeParams& p, int ev, uint3
   if (p.trace && blockIdx.x < 2 && it < kTrMax) p.trace[(blockIdx.x * kTrNum + ev) * kTrMax + it] = clock64();
 }
 #define MLA_TR(ev, it) trace_stamp(p, ev, it)
+// Global-timer stamps of every CTA (entry, after the dependency wait, end) after the per-block
+// area: p.trace[2*kTrNum*kTrMax + 3*cta + k].
+__device__ __forceinline__ void trace_cta(const DecodeParams& p, int k) {
+  if (p.trace && threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    p.trace[2 * kTrNum * kTrMax + 3 * blockIdx.x + k] = static_cast<long long>(t);
+    p.trace[2 * kTrNum * kTrMax + 3 * 4096 + 3 * blockIdx.x + k] = clock64();
+    if (k == 0) {
+      unsigned int smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      p.trace[2 * kTrNum * kTrMax + 6 * 4096 + blockIdx.x] = smid;
+    }
+  }
+}
+#define MLA_TR_CTA(k) trace_cta(p, k)
 #else
+#define MLA_TR_CTA(k) ((void)0)
 #define MLA_TR(ev, it) ((void)0)
 #endif
 

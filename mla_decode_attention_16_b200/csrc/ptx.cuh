@@ -226,6 +226,16 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       : "memory");
 }
 // Arrive once on `bar` when every tcgen05 async op issued so far by this thread completes.
+// Weight-stationary form (M = 32 / 64 / 128): with M = 32 the D tile of N columns is spread over
+// the four TMEM lane quadrants, quadrant q holding rows 0..31 in its lanes and the columns
+// [q*N/4, (q+1)*N/4) of D in N/4 TMEM columns.
+__device__ __forceinline__ void umma_ws_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.ws.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");

@@ -205,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  MLA_TR_CTA(0);
   const uint32_t crank = cluster_ctarank();
   const uint32_t peer = crank ^ 1u;
   const int pair = blockIdx.x >> 1;
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // scheduler): everything above overlapped it; nothing it wrote is read before this wait
   pdl_wait_primary();
   if (threadIdx.x == 0) pdl_launch_dependents();
+  MLA_TR_CTA(1);
 
   const int* meta = p.meta + part * kMetaInts;
   const int R = p.rows;
@@ -735,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ------------------------------------------------------------ teardown
+  MLA_TR_CTA(2);
   __syncwarp();  // lanes of the producer / MMA warps rejoin their elected lane
   tc_fence_before();
   __syncthreads();

@@ -8,25 +8,29 @@
 // With <= 32 query rows the decode is bound by HBM (the cost model of
 // 计算边界特性与优化方向抉择: intensity ~ 2 * h_q * s_q FLOP/B), so the goal is
 // to stream pages at full bandwidth with one CTA per SM and no traffic between
-// SMs.  A 128 x 512 fp32 output would not fit TMEM next to the scores, so the
-// value product is computed transposed:
-//   S   [rows x 64 keys] = Q . K^T      (M = 128 lanes, A = Q resident in TMEM,
-//                                        B = the page's key box in smem)
-//   O^T [512 x rows]   += V^T . P^T     (4 tiles of M = 128 d_v rows, N = NP;
-//                                        A = MN-major view of the page's first
-//                                        8 column boxes, B = P row-major in smem)
-// TMEM: O^T (two buffers of 4*NP columns when NP = 16, one when NP = 32),
-// S 64 columns, Q 288 columns (576 16-bit values per row).  Q of even chunks
-// lives in lane quadrant 0 and of odd chunks in quadrant 1, so the next
-// chunk's Q is written while the current chunk runs (the MMA computes all 128
-// lanes; rows outside the current quadrant are ignored).
+// SMs.  Per 64-token page:
+//   S [rows x 64 keys] = Q . K^T       (M = 128 lanes, A = Q resident in TMEM,
+//                                       B = the page's key box in smem; 36 MMAs)
+//   O [rows x 512]    += P . V         (weight-stationary MMA, M = 32 rows,
+//                                       N = 256 values per half, A = P in smem,
+//                                       B = MN-major view of the page's first 8
+//                                       column boxes; 8 MMAs)
+// Every tcgen05.mma up to N = 128 costs the same ~70 cycles, so the instruction
+// count bounds this kernel: the M = 32 form does P.V in 8 instructions of ~87
+// cycles where 4 tiles of transposed M = 128 products take 16 of ~82.  With
+// M = 32 the output sits in 128 TMEM columns over all four lane quadrants
+// (lane r of quadrant q: row r, values 256h + 64q .. +63 of half h).
+// TMEM: O 128 columns, S 64 columns, Q 288 columns (576 16-bit values per
+// row).  Q of even chunks lives in lane quadrant 0 and of odd chunks in
+// quadrant 1, so the next chunk's Q is written while the current chunk runs
+// (the Q.K^T MMA computes all 128 lanes; rows outside the current quadrant are
+// ignored).
 //
 // Roles (384 threads): warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0
 // issues every tcgen05.mma; warps 4-7: warp 4 + (chunk & 1) runs the softmax
-// of a chunk (one thread per query row) and all four rescale O^T when a row's
-// exponent reference moves; warps 8-11 write each chunk's epilogue from its
-// O^T buffer while the next chunk runs, and warps 8 / 9 load Q for even / odd
-// chunks.
+// of a chunk (one thread per query row) and all four rescale O when a row's
+// exponent reference moves; warps 8-11 write each chunk's epilogue, and warps
+// 8 / 9 load Q for even / odd chunks.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -59,8 +63,8 @@ enum Bar {
   kPFull,                       // [2]
   kPEmpty = kPFull + 2,         // [2]
   kODone = kPEmpty + 2,         // one phase per PV
-  kOFinal,                      // [2] one phase per chunk using that O^T buffer
-  kOEmpty = kOFinal + 2,        // [2] epilogue finished reading that O^T buffer
+  kOFinal,                      // [2] one phase per chunk using that O buffer
+  kOEmpty = kOFinal + 2,        // [2] epilogue finished reading that O buffer
   kStats = kOEmpty + 2,         // [2] row sums / reference maxima of a chunk parity in smem
   kDrain = kStats + 2,
   kNumBars
@@ -68,29 +72,23 @@ enum Bar {
 
 template <int NP>
 struct Layout {
-  static constexpr int kOBufs = NP == 16 ? 2 : 1;
+  static constexpr int kOBufs = 1;
   static constexpr int kOffK = 0;
   static constexpr int kOffP = kOffK + kStages * kStageBytes;  // 1024-aligned
-  static constexpr int kPBytes = NP * 128;                     // P: NP rows x 64 keys (16-bit)
+  static constexpr int kPBytes = 32 * 128;                     // P: 32 rows (M of the P.V MMA) x 64 keys
   static constexpr int kOffRed = kOffP + 2 * kPBytes;
   // floats: alpha [2][NP], flag [2], row sums [2][NP], reference max [2][NP]
   static constexpr int kRedFloats = 2 * NP + 2 + 2 * NP + 2 * NP;
   static constexpr int kOffBar = (kOffRed + kRedFloats * 4 + 7) / 8 * 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = kOBufs * 4 * NP;
+  static constexpr uint32_t kColO = 0;     // O: 2 halves of 256 values x 64 columns (see umma_ws_ss)
+  static constexpr uint32_t kColS = kColO + kOBufs * 128;
   static constexpr uint32_t kColQ = kColS + kPage;
   static_assert(kColQ + kQCols <= kTmemCols, "TMEM budget");
 };
-
-template <bool kBF16>
-__device__ __forceinline__ void store_out(void* out, int64_t idx, float v) {
-  if constexpr (kBF16)
-    reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
-  else
-    reinterpret_cast<__half*>(out)[idx] = __float2half_rn(v);
-}
 
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -101,21 +99,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
   }
-}
-
-template <int NP>
-__device__ __forceinline__ void tmem_ld_np(uint32_t taddr, uint32_t (&r)[NP]) {
-  if constexpr (NP == 16)
-    tmem_ld16(taddr, r);
-  else
-    tmem_ld32(taddr, r);
-}
-template <int NP>
-__device__ __forceinline__ void tmem_st_np(uint32_t taddr, const uint32_t (&r)[NP]) {
-  if constexpr (NP == 16)
-    tmem_st16(taddr, r);
-  else
-    tmem_st32(taddr, r);
 }
 
 // One chunk of a partition: blocks [lo, hi) of request req (n blocks in all).
@@ -158,6 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  MLA_TR_CTA(0);
   const int part = blockIdx.x;
 
   if (threadIdx.x == 0) {
@@ -181,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // scheduler): the prologue above overlapped it; nothing it wrote is read before this wait
   pdl_wait_primary();
   if (threadIdx.x == 0) pdl_launch_dependents();
+  MLA_TR_CTA(1);
 
   const int* meta = p.meta + part * kMetaInts;
   const int br = meta[0], bk = meta[1], er = meta[2], ek = meta[3], bs = meta[4];
@@ -220,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, kPage, false, false);
-      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 128, NP, true, false);
+      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 32, 256, false, true);
       uint32_t it = 0, chunk = 0;
       auto issue_pv = [&](uint32_t itp, int jjp, bool last) {
         const int st = itp % kStages;
@@ -232,14 +217,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         MLA_TR(kTrPv, itp);
         const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
         const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
-        const uint32_t dcol = tmem + ob * 4 * NP;
-#pragma unroll 1
-        for (int m = 0; m < 4; ++m) {
+        const uint32_t dcol = tmem + Lay::kColO + ob * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
           for (int kk = 0; kk < kPage / 16; ++kk) {
-            // V^T rows m*128 .. m*128+127 = column boxes 2m, 2m+1 (8 KB apart); keys 16kk .. 16kk+15
-            const uint64_t adesc = smem_desc_sw128(kst + (2 * m) * kKBox + kk * 2048, kKBox, 1024);
-            const uint64_t bdesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
-            umma_ss(dcol + m * NP, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
+            // O[:, 256h ..] += P[:, 16kk ..] . V[16kk .., 256h ..]: A = P (32 rows, K-major), B = V
+            // (MN-major view of column boxes 4h .. 4h+3, 8 KB apart; 16 keys = 2 x 1 KB)
+            const uint64_t adesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(kst + (4 * h) * kKBox + kk * 2048, kKBox, 1024);
+            umma_ws_ss(dcol + 64 * h, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
           }
         }
         umma_commit(bar(kKvEmpty + st));
@@ -282,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(bar(kDrain), 0);
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ softmax (one warp per chunk) + O^T rescale
+    // ------------------------------------------------------------ softmax (one warp per chunk) + O rescale
     const int q4 = warp & 3;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int r = lane;
@@ -372,15 +359,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kODone), (itc - 1) & 1, abort_flag, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
+          // lane r of every quadrant holds row r: 64 columns of each half of its values
+          const float a = r < NP ? s_alpha[b * NP + r] : 1.f;
 #pragma unroll 1
-          for (int mt = 0; mt < 4; ++mt) {
-            uint32_t o[NP];
-            const uint32_t col = ob * 4 * NP + mt * NP;
-            tmem_ld_np<NP>(t_lane + col, o);
+          for (int c32 = 0; c32 < 4; ++c32) {
+            uint32_t o[32];
+            const uint32_t col = Lay::kColO + ob * 128 + 32 * c32;
+            tmem_ld32(t_lane + col, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < NP; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * s_alpha[b * NP + c]);
-            tmem_st_np<NP>(t_lane + col, o);
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * a);
+            tmem_st32(t_lane + col, o);
           }
           tmem_wait_st();
         }
@@ -389,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(bar(kPFull + b));
       }
       if (smx) {
-        // this stats slot was last used by chunk - 2; with two O^T buffers its epilogue may still
+        // this stats slot was last used by chunk - 2; with two O buffers its epilogue may still
         // be reading it (with one buffer the MMA order already guarantees it finished)
         if (kOBufs == 2 && chunk >= 2)
           mbar_wait(bar(kOEmpty + par), ((chunk >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
@@ -444,21 +433,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool whole = (c.lo == 0 && c.hi == c.n);
       const int64_t chunk0 = whole ? 0 : static_cast<int64_t>(p.num_splits[c.req] + c.split) * R;
       const float* ls = s_lsum + par * NP;
+      // lane r of quadrant q4 holds row r, values 256h + 64 q4 + (0..63) of each half h
+      const float lr = r < NP ? ls[r] : 0.f;
+      const float inv = lr > 0.f ? 1.f / lr : 0.f;
 #pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        uint32_t o[NP];
-        tmem_ld_np<NP>(t_lane + ob * 4 * NP + mt * NP, o);
+      for (int c32 = 0; c32 < 4; ++c32) {
+        uint32_t o[32];
+        tmem_ld32(t_lane + Lay::kColO + ob * 128 + 32 * c32, o);
         tmem_wait_ld();
-        const int d = mt * 128 + q4 * 32 + lane;
+        if (r < R) {
+          const int d = (c32 >> 1) * 256 + q4 * 64 + (c32 & 1) * 32;
+          if (whole) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                                  (static_cast<int64_t>(c.req) * R + r) * kDV + d);
 #pragma unroll
-        for (int cc = 0; cc < NP; ++cc) {
-          if (cc < R) {
-            const float lc = ls[cc];
-            const float v = lc > 0.f ? __uint_as_float(o[cc]) / lc : 0.f;
-            if (whole)
-              store_out<kBF16>(p.out, (static_cast<int64_t>(c.req) * R + cc) * kDV + d, v);
-            else
-              p.o_acc[(chunk0 + cc) * kDV + d] = v;
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack2<kBF16>(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+              w.y = pack2<kBF16>(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+              w.z = pack2<kBF16>(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+              w.w = pack2<kBF16>(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+              dst[v] = w;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.o_acc + (chunk0 + r) * kDV + d);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                   __uint_as_float(o[4 * v + 2]) * inv, __uint_as_float(o[4 * v + 3]) * inv);
           }
         }
       }
@@ -494,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
+  MLA_TR_CTA(2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
