@@ -24,6 +24,11 @@ SMALL = [
     (5, 1, 1, [17, 64, 65, 128, 129], torch.bfloat16, False, 2, 8),  # one query row
     (2, 2, 100, [300, 77], torch.bfloat16, True, None, 9),        # ragged second row tile (200 rows)
     (3, 1, 32, [4096, 1, 2000], torch.float16, False, None, 10),
+    (2, 1, 33, [300, 64], torch.bfloat16, False, None, 11),       # 33 rows: pair kernel, 2 quadrants idle
+    (2, 2, 16, [100, 500], torch.bfloat16, True, None, 12),       # 32 rows, causal: narrow kernel at N = 32
+    (1, 8, 128, [700], torch.bfloat16, True, None, 13),           # 1024 rows (the maximum): 8 row tiles
+    (600, 1, 16, [(37 * i) % 211 for i in range(600)], torch.bfloat16, False, None, 14),  # many short requests
+    (300, 1, 128, [(53 * i) % 307 for i in range(300)], torch.float16, False, None, 15),
 ]
 
 
@@ -50,7 +55,9 @@ def test_tiny_workload():
 def test_metadata_bit_exact():
     import mla_decode_attention_16_b200 as mla
     rng = random.Random(7)
-    cases = [([192, 640, 1, 0, 130], 3), ([4096] * 64, 74), ([4096] * 128, 74), ([0, 0, 0], 5), ([1], 148)]
+    cases = [([192, 640, 1, 0, 130], 3), ([4096] * 64, 74), ([4096] * 128, 74), ([0, 0, 0], 5), ([1], 148),
+             ([rng.randint(0, 3000) for _ in range(16384)], 148),   # the largest batch
+             ([rng.randint(0, 3000) for _ in range(2000)], 1024)]   # the most partitions
     for _ in range(20):
         b = rng.choice([1, 3, 16, 132, 500])
         cases.append(([rng.choice([0, 1, 64, 65, rng.randint(1, 40000)]) for _ in range(b)],
