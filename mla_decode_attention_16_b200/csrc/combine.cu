@@ -48,6 +48,9 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const DecodeParams
   const int b = blockIdx.y;
   const int row = blockIdx.x * kWarps + warp;
   const int R = p.rows;
+  // The next kernel in the stream (normally the next decode's scheduler, which waits for this grid
+  // before writing anything this one reads) may launch now.
+  ptx::pdl_launch_dependents();
   // Everything read here (partials, and num_splits from the scheduler two launches back, which the
   // split-KV kernel itself waited for) is complete and visible once the split-KV grid is.
   ptx::pdl_wait_primary();

@@ -73,6 +73,9 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
   __shared__ long long s_warp[kWarps + 1];
   // the split-KV kernel that follows may start its prologue now; it waits for this grid before reading
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // This kernel is itself launched as a programmatic dependent (normally of the previous decode's
+  // combine kernel): it reads only the lengths before the wait below, and writes its outputs, which
+  // the previous decode's kernels read, only after it.
 
   for (int i = threadIdx.x; i < batch; i += kThreads) {
     const int L = seqlens[i];
@@ -95,6 +98,7 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
   }
   __syncthreads();
   const long long total_pieces = block_exclusive_scan(s_cnt, batch, s_warp);
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernels in the stream are done
   for (int i = threadIdx.x; i < batch; i += kThreads) num_splits[i] = s_cnt[i];
   if (threadIdx.x == 0) num_splits[batch] = static_cast<int32_t>(total_pieces);
 
@@ -145,9 +149,17 @@ const void* metadata_kernel_ptr() { return reinterpret_cast<const void*>(&metada
 
 cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, int32_t* meta, int32_t* num_splits,
                             cudaStream_t stream) {
-  metadata::metadata_kernel<<<1, metadata::kThreads, metadata_smem_bytes(batch, num_parts), stream>>>(
-      seqlens, batch, num_parts, meta, num_splits);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(metadata::kThreads);
+  cfg.dynamicSmemBytes = metadata_smem_bytes(batch, num_parts);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, metadata::metadata_kernel, seqlens, batch, num_parts, meta, num_splits);
 }
 
 }  // namespace mla

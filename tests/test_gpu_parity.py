@@ -29,6 +29,7 @@ SMALL = [
     (1, 8, 128, [700], torch.bfloat16, True, None, 13),           # 1024 rows (the maximum): 8 row tiles
     (600, 1, 16, [(37 * i) % 211 for i in range(600)], torch.bfloat16, False, None, 14),  # many short requests
     (300, 1, 128, [(53 * i) % 307 for i in range(300)], torch.float16, False, None, 15),
+    (4, 1, 64, [0, 5, 0, 640], torch.bfloat16, False, 3, 16),      # pair kernel: empty requests, splits
 ]
 
 
