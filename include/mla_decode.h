@@ -78,9 +78,10 @@ int mla_version(void);
 
 /*
  * Number of scheduler partitions for `rows` = s_q * h_q query rows per request
- * on `device` (one partition = one CTA pair per 128-row tile).  Host only; it
- * queries the device's SM count and cluster occupancy once and caches it.
- * rows must be in [1, 1024].
+ * on `device`: one per SM when rows <= 32 (one CTA per partition), else the
+ * number of co-resident CTA pairs divided by the number of 128-row tiles (one
+ * CTA pair per partition and tile).  Host only; it queries the device's SM
+ * count and cluster occupancy once and caches it.  rows must be in [1, 1024].
  */
 int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts);
 
@@ -112,14 +113,21 @@ int mla_get_workspace_size(int batch, int rows, int num_sm_parts, size_t* bytes)
  * so its work (blocks + 5 per piece) is at most S + 5, the walk-through's
  * ceil_div(total, num_sm_parts) + fixed overhead.
  * Enqueues one single-CTA kernel on `stream` (data-parallel: prefix sums and
- * one binary search per partition).
+ * one binary search per partition) as a programmatic dependent launch: it may
+ * start while the previous kernel in the stream finishes, reads cache_seqlens
+ * right away, and writes its two outputs only after that kernel has completed.
+ * So cache_seqlens must be final before the previous kernel lets dependents
+ * start early (kernels that do not use programmatic dependent launch let them
+ * start only when they complete; this library's combine kernel lets them
+ * start at once and never writes cache_seqlens).
  */
 int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows, int num_sm_parts,
                      int32_t* tile_sched_metadata, int32_t* num_splits, void* stream);
 
 /*
- * Decode forward: split-KV kernel, then (programmatic dependent launch) the
- * log-sum-exp combine kernel.
+ * Decode forward: split-KV kernel, then the log-sum-exp combine kernel, each a
+ * programmatic dependent launch of the kernel before it (it sets up while that
+ * kernel finishes and waits for it before reading anything it wrote).
  *   q                 device [batch, s_q, h_q, 576], dtype, contiguous, 16-B aligned
  *   kcache            device [num_pages, 64, 1, 576], dtype, contiguous, 16-B aligned
  *   num_pages         pages in kcache (>= 1)
