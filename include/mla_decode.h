@@ -52,7 +52,7 @@ extern "C" {
 #define MLA_HEAD_DIM_V 512
 #define MLA_PAGE_SIZE 64
 #define MLA_META_INTS 8
-#define MLA_FIXED_OVERHEAD_BLOCKS 5
+#define MLA_FIXED_OVERHEAD_BLOCKS 3
 
 #define MLA_DEVERR_TIMEOUT 1
 #define MLA_DEVERR_PAGE_INDEX 2
@@ -108,9 +108,10 @@ int mla_get_workspace_size(int batch, int rows, int num_sm_parts, size_t* bytes)
  *   num_splits           device int32 [batch + 1], written: prefix sums of the
  *                        number of chunks each request is cut into
  * Blocks n_b = ceil(L_b / 64).  Requests are laid end to end on a line of
- * units (5 units of fixed overhead, then one unit per block); with the share
- * S = ceil(sum_{n_b>0}(n_b + 5) / P), partition p owns units [p*S, (p+1)*S),
- * so its work (blocks + 5 per piece) is at most S + 5, the walk-through's
+ * units (F = MLA_FIXED_OVERHEAD_BLOCKS = 3 units of fixed overhead, then one
+ * unit per block); with the share S = ceil(sum_{n_b>0}(n_b + F) / P),
+ * partition p owns units [p*S, (p+1)*S), so its work (blocks + F per piece)
+ * is at most S + F, the walk-through's
  * ceil_div(total, num_sm_parts) + fixed overhead.
  * Enqueues one single-CTA kernel on `stream` (data-parallel: prefix sums and
  * one binary search per partition) as a programmatic dependent launch: it may

@@ -2,8 +2,10 @@
 // "FlashMLA 在 Hopper GPU 上的 MHA 内核调度优化解析", 辅助优化：可编程依赖启动与瓦片调度).
 //
 // Every request is n_b = ceil(L_b / 64) blocks of 64 tokens, and each piece of
-// work on a request costs a fixed overhead of F = 5 blocks (Q load, pipeline
-// fill, epilogue, merge).  The requests are laid end to end on a line of
+// work on a request costs a fixed overhead of F = 3 blocks (Q load, pipeline
+// fill, epilogue, merge; on B200 a second piece in a partition measured about
+// one block of extra time, and F = 3 gave the shortest memory-bound launches
+// of F = 1, 3, 5, 8, 12).  The requests are laid end to end on a line of
 // units -- F overhead units, then one unit per block -- and partition p of P
 // owns the units [p*S, (p+1)*S) with the share S = ceil(total / P), so block k
 // of request b belongs to partition (cum_b + F + k) / S.  A partition's work is

@@ -17,8 +17,10 @@ Sources:
 
 Reading (the pages give the share formula, not the assignment; listed in
 DESIGN.md):
-* n_r = ceil(L_r / 64) blocks per request; F = 5 units of fixed overhead per
-  request that has blocks.  Requests are laid end to end on a line of units:
+* n_r = ceil(L_r / 64) blocks per request; F = 3 units of fixed overhead per
+  request that has blocks.  The pages name fixed_overhead_num_blocks without a
+  value; F is a tuning constant of the scheduler (every F gives a valid
+  schedule with the bounds below), set to the value the device library uses.  Requests are laid end to end on a line of units:
   request r occupies F overhead units followed by its n_r block units, so its
   block k sits at unit x = cum_r + F + k, where cum_r is the sum of (F + n_t)
   over the non-empty requests t < r.  total = sum over non-empty requests of
@@ -46,7 +48,7 @@ from __future__ import annotations
 from typing import Dict, List, Sequence, Tuple
 
 PAGE_BLOCK = 64
-FIXED_OVERHEAD_BLOCKS = 5
+FIXED_OVERHEAD_BLOCKS = 3
 META_INTS = 8
 
 
