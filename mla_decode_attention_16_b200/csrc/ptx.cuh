@@ -167,6 +167,13 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t remot
       : "memory");
 }
 
+// 4-byte store into a peer CTA's shared memory that completes 4 bytes on the peer's mbarrier.
+__device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t remote_bar, float v) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to a peer
 // CTA's shared memory; completes `bytes` on the peer's mbarrier.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
@@ -181,6 +188,11 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // Wait until every committed bulk copy of this thread has finished reading its source.
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// ... all but the N most recently committed groups.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
 // ----------------------------------------------------------------- PDL
@@ -344,6 +356,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t smem_addr, uint32_t 
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(4) << 61;
+  return d;
+}
+
+// Same with 32-byte swizzling (mode 6): K-major rows of 32 bytes, 8-row atoms of 256 bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(6) << 61;
   return d;
 }
 

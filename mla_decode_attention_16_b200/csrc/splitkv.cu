@@ -18,31 +18,36 @@
 //    32 columns 512 + 32c ..  Those 256 main columns of Q stay in TMEM for the
 //    whole chunk (A operand from TMEM); the 32 others come from a
 //    shared-memory box.
-//  * The partial scores of a 64-key block are exchanged between the pair
-//    through distributed shared memory: rounded to 24 bits (sign, exponent, 15
-//    mantissa bits), staged, and moved by one bulk copy per warp that completes
-//    on the peer's mbarrier.  Both CTAs round both partials the same way, so
-//    they hold bit-identical scores and run the same softmax; their two O
-//    halves stay consistent.
-//  * The exchange runs one block ahead: right after combining block t, each
-//    softmax warp sends its partial of block t+1, which travels while block t's
-//    probabilities are computed.  A warp signals "slot consumed" with a relaxed
-//    arrive whose input depends on every word it read (a cluster-scope release
-//    there cost ~1000 cycles per block).
+//  * The softmax of a 64-key block is split between the pair by key: CTA c
+//    exponentiates keys 32c .. 32c+31 of every row.  It sends its partial
+//    scores of the other 32 keys to the peer, rounded to 24 bits (sign,
+//    exponent, 15 mantissa bits) and moved by one bulk copy per warp that
+//    completes on the peer's mbarrier, and receives the peer's partials of its
+//    own keys.  The two CTAs share each row's block maximum (distributed
+//    shared memory stores) so they keep the same exponent reference, and each
+//    copies the P of its keys into the peer's P, so both P.V products see the
+//    whole block; the row sums are added at the end of a chunk.
+//  * The score exchange runs one block ahead: while block t's maximum travels,
+//    each softmax warp sends its partial of block t+1.  A warp signals "slot
+//    consumed" with a relaxed arrive whose input depends on every word it read
+//    (a cluster-scope release there cost ~1000 cycles per block).
 //  * Each CTA TMA-loads, per page, four 64-column boxes (128-byte swizzle) at
 //    columns 256c + 64i -- also this CTA's V half -- and one 32-column box
 //    (64-byte swizzle) at 512 + 32c: 36 KB per page, four page stages, so the
 //    HBM latency of a page load hides behind three blocks of work; EVICT_FIRST
 //    L2 policy on page loads (细粒度流水线与缓存优化).
-//  * P goes to shared memory (K-major A operand of PV; V is the MN-major B
-//    operand read straight from the page tile).
+//  * P goes to shared memory as four K-major tiles of 16 keys with 32-byte
+//    swizzle (the A operand of the four K = 16 steps of PV), so the piece one
+//    warp writes -- 32 rows x 16 keys -- is one contiguous kilobyte that a
+//    single bulk copy puts into the peer's P; V is the MN-major B operand read
+//    straight from the page tile.
 //  * Roles: warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0 issues every
 //    tcgen05.mma (Q.K^T two blocks ahead of P.V); warps 4-11 two per TMEM lane
-//    quadrant, one thread per (query row, half of the block's 64 keys): Q into
+//    quadrant, one thread per (query row, 16 of its CTA's 32 keys): Q into
 //    TMEM, score exchange, softmax (exp2 with log2(e) folded into the scale,
 //    "FlashMLA: 高性能GPU注意力机制计算库" 4. Softmax数值稳定性优化), O correction,
-//    epilogue.  The two threads of a row agree on its maximum through shared
-//    memory and keep separate partial row sums, added at the end of a chunk.
+//    epilogue.  The four threads of a row (two per CTA) agree on its maximum
+//    and keep separate partial row sums, added at the end of a chunk.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -64,22 +69,24 @@ constexpr int kKBox = kBlockN * 128;        // 8 KB: 64 keys x 64 columns (128-b
 constexpr int kKrBox = kBlockN * 64;        // 4 KB: 64 keys x 32 columns (64-byte swizzle)
 constexpr int kStageBytes = 4 * kKBox + kKrBox;  // 36 KB
 constexpr int kStages = 4;
-constexpr int kPBytes = kTileRows * 128;    // 16 KB: P, 128 rows x 64 keys (16-bit)
-constexpr int kSmWarps = 8;                 // softmax warps: 4 lane quadrants x 2 key halves
-constexpr int kHalfN = kBlockN / 2;         // keys per softmax thread
-constexpr int kRowWords = kHalfN * 3 / 4;   // 24 words: 32 scores at 24 bits
-constexpr int kRowBytes = kRowWords * 4;    // 96
-constexpr int kXWarp = 32 * kRowBytes;      // 3 KB per warp and direction
-constexpr int kXBytes = kSmWarps * kXWarp;  // 24 KB
+constexpr int kPTile = kTileRows * 32;      // 4 KB: P of 16 keys x 128 rows (16-bit, 32-byte swizzle)
+constexpr int kPBytes = 4 * kPTile;         // 16 KB: the block's 64 keys
+constexpr int kSmWarps = 8;                 // softmax warps: 4 lane quadrants x 2 key quarters
+constexpr int kOwnN = kBlockN / 4;          // 16 keys per softmax thread
+constexpr int kRowWords = kOwnN * 3 / 4;    // 12 words: 16 scores at 24 bits
+constexpr int kRowBytes = kRowWords * 4;    // 48
+constexpr int kXWarp = 32 * kRowBytes;      // 1.5 KB per warp and direction
+constexpr int kXBytes = kSmWarps * kXWarp;  // 12 KB
+constexpr int kSlotFloats = 2 * 2 * 2 * kTileRows;  // row values: [parity][source CTA][key quarter][row]
 
 constexpr int kOffQR = 0;                               // this CTA's 32 of Q's columns 512..575
 constexpr int kOffK = kOffQR + kQrBox;                  // page stages
 constexpr int kOffP = kOffK + kStages * kStageBytes;    // P
 constexpr int kOffStg = kOffP + kPBytes;                // send staging [8 warps]
 constexpr int kOffRcv = kOffStg + kXBytes;              // receive [8 warps]
-constexpr int kOffRed = kOffRcv + kXBytes;              // row maxima / sums [2 parities][2 halves][128 rows]
+constexpr int kOffRed = kOffRcv + kXBytes;              // row maxima / sums of both CTAs
 static_assert(kOffK % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "swizzle atom alignment");
-constexpr int kOffBar = kOffRed + 2 * 2 * kTileRows * 4;
+constexpr int kOffBar = kOffRed + kSlotFloats * 4;
 
 enum Bar {
   kKvFull = 0,
@@ -89,14 +96,15 @@ enum Bar {
   kQEmpty,                       // the chunk's last Q.K^T completed
   kSFull,                        // [2]
   kSEmpty = kSFull + 2,          // [2], 8 warps
-  kPFull = kSEmpty + 2,          // 8 warps, one phase per block
+  kPFull = kSEmpty + 2,          // 8 warps + the peer's copies of its P, one phase per block
   kPEmpty,                       // one phase per P.V
   kOFinal,                       // one phase per chunk: its last P.V completed
   kOEmpty,                       // 8 warps, one phase per chunk
   kXFull,                        // [8 warps]: the peer's partial landed
   kXEmpty = kXFull + kSmWarps,   // [8 warps]: the peer consumed what this CTA sent
-  kRowX = kXEmpty + kSmWarps,    // [4 quadrants]: the two warps of a quadrant swap row values
-  kDrain = kRowX + 4,
+  kXchg = kXEmpty + kSmWarps,    // [4 quadrants][2 parities]: the row values of both CTAs are in
+  kPeerFree = kXchg + 8,         // [8 warps]: the peer's P.V of the previous block completed
+  kDrain = kPeerFree + kSmWarps,
   kNumBars
 };
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -215,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
       const bool eight = i == kQtFull || i == kSEmpty || i == kSEmpty + 1 || i == kPFull || i == kOEmpty;
-      const bool two = i >= kRowX && i < kRowX + 4;
+      const bool two = i >= kXchg && i < kXchg + 8;
       mbar_init(bar(i), eight ? static_cast<uint32_t>(kSmWarps) : two ? 2u : 1u);
     }
     *abort_flag = 0;
@@ -339,8 +347,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vbase = sbase + kOffK + st * kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          // P columns 16kk.. (K-major, 128 rows); V rows 16kk.. (MN-major: 64-column boxes 8 KB apart)
-          const uint64_t adesc = smem_desc_sw128(sbase + kOffP + kk * 32, 16, 1024);
+          // P keys 16kk.. (tile kk: K-major, 128 rows of 32 bytes); V rows 16kk.. (MN-major: 64-column
+          // boxes 8 KB apart)
+          const uint64_t adesc = smem_desc_sw32(sbase + kOffP + kk * kPTile, 16, 256);
           const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, kKBox, 1024);
           umma_ss(tmem + kColO, adesc, bdesc, idesc_pv, (!wp.first() || kk > 0) ? 1u : 0u);
         }
@@ -380,37 +389,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ Q to TMEM, exchange, softmax, correction, epilogue
-    // Two warps per TMEM lane quadrant: warp 4 + q4 takes keys 0..31 of its 32 rows, warp 8 + q4
-    // keys 32..63; both keep the same row maximum (shared through shared memory).
+    // Two warps per TMEM lane quadrant.  Of the block's 64 keys this CTA exponentiates 32c ..
+    // 32c+31: warp 4 + q4 the first 16 of its 32 rows, warp 8 + q4 the last 16.  Each warp also
+    // sends the peer its partial scores of keys 32p + 16 sub .. (p = the peer's rank).
     const int sm = warp - 4;          // 0..7
     const int q4 = warp & 3;
-    const int half = sm >> 2;
+    const int sub = sm >> 2;          // which 16 of the CTA's 32 keys
     const int row = q4 * 32 + lane;
     const int row_g = mtile * kTileRows + row;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const int own_col = 32 * static_cast<int>(crank) + kOwnN * sub;   // S columns this thread exponentiates
+    const int send_col = 32 * static_cast<int>(peer) + kOwnN * sub;   // S columns it sends to the peer
+    // its P: tile 2c + sub (keys own_col ..), rows 32 q4 .. 32 q4 + 31 = one contiguous kilobyte
+    const uint32_t p_piece = sbase + kOffP + (2 * crank + sub) * kPTile + q4 * 32 * 32;
     uint8_t* stg_row = smem + kOffStg + sm * kXWarp + lane * kRowBytes;
     const uint32_t stg_warp = sbase + kOffStg + sm * kXWarp;
-    float* red = reinterpret_cast<float*>(smem + kOffRed);  // [parity][half][row]
-    uint32_t rx_phase = 0;
-    // the other half's value of this row (both halves call it with their own): one phase of the
-    // quadrant's barrier per swap; the two parities of the buffer keep a fast half's next write
-    // off the slot the other half may still be reading (it cannot write twice ahead: the swap
-    // after next waits for the other half's arrival of the next one)
-    auto row_swap = [&](float v) {
-      float* slot = red + (rx_phase & 1) * 2 * kTileRows;
-      slot[half * kTileRows + row] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kRowX + q4));
-      mbar_wait(bar(kRowX + q4), rx_phase & 1, abort_flag, err, kDevErrTimeout);
-      const float o = slot[(half ^ 1) * kTileRows + row];
-      ++rx_phase;
-      return o;
-    };
-    // 16-byte chunk order within a 96-byte row: lanes i and i+4 of each group of 8 differ
-    const int sw = (lane >> 2) & 1;
+    float* slots = reinterpret_cast<float*>(smem + kOffRed);  // [parity][source CTA][key quarter][row]
     // a quadrant whose 32 rows are all padding keeps the barrier protocol but skips the math;
     // its peer quadrant skips the same way
     const bool active = mtile * kTileRows + q4 * 32 < R;
+    const int active_quadrants = min(4, (R - mtile * kTileRows + 31) / 32);
 #ifdef MLA_TRACE
     // developer builds: cycles spent per section, summed over the blocks
     long long tr_acc[kTrNum] = {};
@@ -425,10 +423,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       (void)ev;
     };
 
-    // Q columns 256c + 128h .. +127 of this thread's row of request `req` -> TMEM columns kColQ + 64h ..
+    // The row's four values of one kind (its block maximum, its row sum), one per thread of the
+    // row in either CTA: post puts this thread's into this CTA's slot and (a 4-byte distributed
+    // shared memory store completing on the peer's barrier) into the peer's; wait returns all four
+    // as v[2 * cta + quarter].  One phase of the quadrant's barrier of parity x & 1 per exchange:
+    // the two local warps arrive, the peer's two warps' stores (2 x 32 x 4 bytes) complete it.  A
+    // slot of parity x & 1 is written again only in exchange x + 2, which on either side follows
+    // this thread's exchange x + 1 and so its reading of exchange x.
+    uint32_t xc = 0;
+    // Lane 0's bulk copies alternate between the partial of a block (staging rows) and the P piece
+    // of a block; before rewriting either source, the copy that last read it must be done, and at
+    // most one copy of the other kind was committed after it.
+    int last_copy = 0;  // 0 none yet, 1 partial, 2 P piece
+    auto xchg_post = [&](float v) {
+      const int par = xc & 1;
+      const uint32_t xb = bar(kXchg + 2 * q4 + par);
+      const int idx = par * 4 * kTileRows + (2 * static_cast<int>(crank) + sub) * kTileRows + row;
+      slots[idx] = v;
+      st_async_b32(mapa(sbase + kOffRed + 4 * idx, peer), mapa(xb, peer), v);
+      __syncwarp();
+      if (lane == 0) {
+        if (sub == 0)
+          mbar_arrive_expect_tx(xb, 2 * 32 * 4);
+        else
+          mbar_arrive(xb);
+      }
+    };
+    auto xchg_wait = [&](float (&v)[4]) {
+      const int par = xc & 1;
+      mbar_wait(bar(kXchg + 2 * q4 + par), (xc >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      const float* slot = slots + par * 4 * kTileRows + row;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = slot[k * kTileRows];
+      ++xc;
+    };
+
+    // Q columns 256c + 128 sub .. +127 of this thread's row of request `req` -> TMEM columns kColQ + 64 sub ..
     auto q_row = [&](int req) {
       return reinterpret_cast<const uint8_t*>(qptr) +
-             ((static_cast<int64_t>(req) * R + (row_g < R ? row_g : 0)) * kDK + 256 * crank + 128 * half) * 2;
+             ((static_cast<int64_t>(req) * R + (row_g < R ? row_g : 0)) * kDK + 256 * crank + 128 * sub) * 2;
     };
     auto prefetch_q = [&](int req) {
       if (row_g >= R) return;
@@ -450,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           w[4 * v + 2] = d.z;
           w[4 * v + 3] = d.w;
         }
-        tmem_st32(t_lane + kColQ + 64 * half + 32 * c32, w);
+        tmem_st32(t_lane + kColQ + 64 * sub + 32 * c32, w);
       }
       tmem_wait_st();
     };
@@ -478,24 +511,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       stamp(kTrSmS, u);
       if (!active) return;
-      uint32_t r[32];
-      tmem_ld32(t_lane + kColS + 64 * b + kHalfN * half, r);
+      uint32_t r[16];
+      tmem_ld16(t_lane + kColS + 64 * b + send_col, r);
       tmem_wait_ld();
       stamp(kTrA, u);
-      if (lane == 0) bulk_wait_read_all();  // the previous copy out of the staging row is done
+      // the previous partial's copy out of the staging rows is done (a P copy committed since may
+      // still be reading)
+      if (lane == 0) {
+        if (last_copy == 2)
+          bulk_wait_read<1>();
+        else
+          bulk_wait_read_all();
+      }
       __syncwarp();
       stamp(kTrB, u);
-#pragma unroll
-      for (int k = 0; k < kRowWords / 12; ++k) {  // 16 scores -> 12 words -> 3 chunks
-        uint32_t w[12];
+      {
+        uint32_t w[kRowWords];  // 16 scores -> 12 words -> 3 chunks (48-byte rows: no bank conflicts)
 #pragma unroll
         for (int g = 0; g < 4; ++g)
-          pack24(r[16 * k + 4 * g], r[16 * k + 4 * g + 1], r[16 * k + 4 * g + 2], r[16 * k + 4 * g + 3], w[3 * g],
-                 w[3 * g + 1], w[3 * g + 2]);
+          pack24(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3], w[3 * g], w[3 * g + 1], w[3 * g + 2]);
 #pragma unroll
         for (int j = 0; j < 3; ++j)
-          *reinterpret_cast<uint4*>(stg_row + (((3 * k + j) ^ sw) << 4)) =
-              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          *reinterpret_cast<uint4*>(stg_row + 16 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
       fence_proxy_async_smem();  // the bulk copy reads the staging through the async proxy
       __syncwarp();
@@ -506,6 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_copy_to_peer(mapa(sbase + kOffRcv + sm * kXWarp, peer), stg_warp, kXWarp, mapa(bar(kXFull + sm), peer));
         bulk_commit_group();
       }
+      last_copy = 1;
       __syncwarp();
       stamp(kTrSend, u);
     };
@@ -522,37 +560,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       wu.next(p);
     }
     uint32_t u = 1;
-    float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: this half's row sum relative to it
+    float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: this thread's keys' row sum relative to it
     for (uint32_t t = 0; wt.valid; ++t, wt.next(p)) {
       if (*abort_flag) break;
       // ---- block t: own partial (rounded as sent) + the peer's, then release the score buffer
       const int b = t & 1;
-      float x[kHalfN];
+      float x[kOwnN];
       if (active) {
         mbar_wait<true>(bar(kXFull + sm), t & 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
         stamp(kTrSmX, t);
-        uint32_t r[32];
-        tmem_ld32(t_lane + kColS + 64 * b + kHalfN * half, r);
+        uint32_t r[16];
+        tmem_ld16(t_lane + kColS + 64 * b + own_col, r);
         tmem_wait_ld();
         stamp(kTrD, t);
         const uint8_t* rcv_row = smem + kOffRcv + sm * kXWarp + lane * kRowBytes;
+        const uint4 c0 = *reinterpret_cast<const uint4*>(rcv_row);
+        const uint4 c1 = *reinterpret_cast<const uint4*>(rcv_row + 16);
+        const uint4 c2 = *reinterpret_cast<const uint4*>(rcv_row + 32);
+        const uint32_t wv[12] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
 #pragma unroll
-        for (int k = 0; k < kRowWords / 12; ++k) {  // 3 chunks = 16 scores per step
-          const uint4 c0 = *reinterpret_cast<const uint4*>(rcv_row + (((3 * k) ^ sw) << 4));
-          const uint4 c1 = *reinterpret_cast<const uint4*>(rcv_row + (((3 * k + 1) ^ sw) << 4));
-          const uint4 c2 = *reinterpret_cast<const uint4*>(rcv_row + (((3 * k + 2) ^ sw) << 4));
-          const uint32_t wv[12] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w, c2.x, c2.y, c2.z, c2.w};
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            float a0, a1, a2, a3;
-            unpack24(wv[3 * g], wv[3 * g + 1], wv[3 * g + 2], a0, a1, a2, a3);
-            const int c = 16 * k + 4 * g;
-            x[c] = round24(r[c]) + a0;
-            x[c + 1] = round24(r[c + 1]) + a1;
-            x[c + 2] = round24(r[c + 2]) + a2;
-            x[c + 3] = round24(r[c + 3]) + a3;
-          }
+        for (int g = 0; g < 4; ++g) {
+          float a0, a1, a2, a3;
+          unpack24(wv[3 * g], wv[3 * g + 1], wv[3 * g + 2], a0, a1, a2, a3);
+          const int c = 4 * g;
+          x[c] = round24(r[c]) + a0;
+          x[c + 1] = round24(r[c + 1]) + a1;
+          x[c + 2] = round24(r[c + 2]) + a2;
+          x[c + 3] = round24(r[c + 3]) + a3;
         }
         stamp(kTrE, t);
       }
@@ -565,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = -INFINITY;
         l = 0.f;
       }
-      float mx = -INFINITY;  // this half's maximum of the block's scaled scores
+      float mx = -INFINITY;  // this thread's maximum of the block's scaled scores
       if (active) {
         // ---- online softmax in log2 units
         int limit = 0;
@@ -573,16 +608,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           limit = p.causal ? wt.L - (p.s_q - 1 - row_g / p.h_q) : wt.L;
           limit = limit < 0 ? 0 : limit;
         }
-        const int kbase = wt.blk * kBlockN + kHalfN * half;
-        if (__all_sync(0xffffffffu, kbase + kHalfN <= limit)) {
+        const int kbase = wt.blk * kBlockN + own_col;
+        if (__all_sync(0xffffffffu, kbase + kOwnN <= limit)) {
 #pragma unroll
-          for (int c = 0; c < kHalfN; ++c) {
+          for (int c = 0; c < kOwnN; ++c) {
             x[c] *= p.scale_log2;
             mx = fmaxf(mx, x[c]);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < kHalfN; ++c) {
+          for (int c = 0; c < kOwnN; ++c) {
             x[c] = (kbase + c < limit) ? x[c] * p.scale_log2 : -INFINITY;
             mx = fmaxf(mx, x[c]);
           }
@@ -596,10 +631,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar(kXFull + sm), kXWarp);
           mbar_arrive_cluster_relaxed_after(mapa(bar(kXEmpty + sm), peer), mx);
         }
-        __syncwarp();
+        xchg_post(mx);
         stamp(kTrQk, t);
       }
-      if (wu.valid) {  // block t + 1's partial travels while block t's softmax runs
+      if (wu.valid) {  // block t + 1's partial travels while block t's maximum does
         send_partial(u, wu);
         wu.next(p);
         ++u;
@@ -607,10 +642,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!active) {
         mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kPFull));
+        if (lane == 0) {
+          if (sm == 0)
+            mbar_arrive_expect_tx(bar(kPFull), active_quadrants * 2 * 1024);
+          else
+            mbar_arrive(bar(kPFull));
+        }
       } else {
-        // both halves of the row take the same maximum
-        mx = fmaxf(mx, row_swap(mx));
+        // the row's maximum over all 64 keys, the same in both CTAs
+        {
+          float v[4];
+          xchg_wait(v);
+          mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+        }
         stamp(kTrG, t);
         bool resc = false;
         float alpha = 1.f;
@@ -623,9 +667,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float base = (m == -INFINITY) ? 0.f : m;
         float s0 = 0.f, s1 = 0.f;
-        uint32_t pk[kHalfN / 2];
+        uint32_t pk[kOwnN / 2];
 #pragma unroll
-        for (int c2 = 0; c2 < kHalfN / 2; ++c2) {
+        for (int c2 = 0; c2 < kOwnN / 2; ++c2) {
           const float p0 = ex2(x[2 * c2] - base);
           const float p1 = ex2(x[2 * c2 + 1] - base);
           s0 += p0;
@@ -635,26 +679,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = l * alpha + (s0 + s1);
         stamp(kTrH, t);
 
-        // P (this half's 32 keys of the row), once the previous P.V has read P (so O also holds
-        // every earlier block)
+        // P (this thread's 16 keys of the row), once this CTA's previous P.V has read P (so O also
+        // holds every earlier block); then tell the peer it may copy its part of P here
         mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        if (lane == 0) {
+          mbar_arrive_cluster_relaxed_after(mapa(bar(kPeerFree + sm), peer), 0.f);
+          // this piece's copy of the previous block is done (a partial's copy may follow it)
+          if (last_copy == 1)
+            bulk_wait_read<1>();
+          else
+            bulk_wait_read_all();
+        }
         __syncwarp();
         tc_fence_after();
         {
-          uint8_t* prow = smem + kOffP + row * 128;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint4*>(prow + (((4 * half + k) ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+          uint8_t* prow = smem + kOffP + (2 * crank + sub) * kPTile + row * 32;
+          const int sw = (row >> 2) & 1;  // 32-byte swizzle: 16-byte chunk index ^ address bit 7
+          *reinterpret_cast<uint4*>(prow + ((0 ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(prow + ((1 ^ sw) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
-        fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+        fence_proxy_async_smem();  // P is read by the tensor core and the bulk copy (async proxy)
+        __syncwarp();
+        if (lane == 0) {
+          // the peer's P.V of the previous block has read its P too
+          mbar_wait<true>(bar(kPeerFree + sm), t & 1, abort_flag, err, kDevErrTimeout);
+          bulk_copy_to_peer(mapa(p_piece, peer), p_piece, 1024, mapa(bar(kPFull), peer));
+          bulk_commit_group();
+        }
+        last_copy = 2;
         if (__any_sync(0xffffffffu, resc)) {
           // only blocks after the chunk's first can move an established reference, so O holds
-          // the chunk's earlier blocks here; each half rescales 128 of the 256 columns
+          // the chunk's earlier blocks here; each warp of the quadrant rescales 128 of the 256 columns
 #pragma unroll 1
           for (int k = 0; k < 4; ++k) {
             uint32_t o[32];
-            const uint32_t ta = t_lane + kColO + 128 * half + 32 * k;
+            const uint32_t ta = t_lane + kColO + 128 * sub + 32 * k;
             tmem_ld32(ta, o);
             tmem_wait_ld();
 #pragma unroll
@@ -665,7 +724,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kPFull));
+        if (lane == 0) {
+          if (sm == 0)
+            mbar_arrive_expect_tx(bar(kPFull), active_quadrants * 2 * 1024);
+          else
+            mbar_arrive(bar(kPFull));
+        }
         __syncwarp();
         stamp(kTrSmP, t);
       }
@@ -674,8 +738,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- epilogue of the chunk: normalise this CTA's O half and write it
       float lt = 0.f;
       if (active) {
-        const float lo = row_swap(l);
-        lt = half == 0 ? l + lo : lo + l;  // same order in both halves
+        float v[4];
+        xchg_post(l);
+        xchg_wait(v);
+        lt = (v[0] + v[1]) + (v[2] + v[3]);  // the same order in both CTAs
       }
       mbar_wait(bar(kOFinal), wt.chunk & 1, abort_flag, err, kDevErrTimeout);
       __syncwarp();
@@ -689,10 +755,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int k = 0; k < 4; ++k) {
           uint32_t o[32];
-          tmem_ld32(t_lane + kColO + 128 * half + 32 * k, o);
+          tmem_ld32(t_lane + kColO + 128 * sub + 32 * k, o);
           tmem_wait_ld();
           if (row_g < R) {
-            const int col = static_cast<int>(crank) * 256 + 128 * half + 32 * k;
+            const int col = static_cast<int>(crank) * 256 + 128 * sub + 32 * k;
             if (whole) {
               uint4* dst = reinterpret_cast<uint4*>(
                   reinterpret_cast<uint16_t*>(p.out) + (static_cast<int64_t>(wt.req) * R + row_g) * kDV + col);
@@ -714,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (crank == 0 && half == 0 && row_g < R) {
+        if (crank == 0 && sub == 0 && row_g < R) {
           const float lse_v = lt > 0.f ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
           if (whole) {
             const int s = row_g / p.h_q, h = row_g % p.h_q;
