@@ -21,9 +21,11 @@
 //  * The softmax of a 64-key block is split between the pair by key: CTA c
 //    exponentiates keys 32c .. 32c+31 of every row.  It sends its partial
 //    scores of the other 32 keys to the peer, rounded to 24 bits (sign,
-//    exponent, 15 mantissa bits) and moved by one bulk copy per warp that
-//    completes on the peer's mbarrier, and receives the peer's partials of its
-//    own keys.  The two CTAs share each row's block maximum (distributed
+//    exponent, 15 mantissa bits) and written by each thread straight from
+//    registers into the peer's shared memory (three 16-byte st.async that
+//    complete on the peer's mbarrier; bulk copies measured slower here, as they
+//    queue in the copy engine behind the page loads), and receives the peer's
+//    partials of its own keys.  The two CTAs share each row's block maximum (distributed
 //    shared memory stores) so they keep the same exponent reference, and each
 //    copies the P of its keys into the peer's P, so both P.V products see the
 //    whole block; the row sums are added at the end of a chunk.
@@ -82,8 +84,7 @@ constexpr int kSlotFloats = 2 * 2 * 2 * kTileRows;  // row values: [parity][sour
 constexpr int kOffQR = 0;                               // this CTA's 32 of Q's columns 512..575
 constexpr int kOffK = kOffQR + kQrBox;                  // page stages
 constexpr int kOffP = kOffK + kStages * kStageBytes;    // P
-constexpr int kOffStg = kOffP + kPBytes;                // send staging [8 warps]
-constexpr int kOffRcv = kOffStg + kXBytes;              // receive [8 warps]
+constexpr int kOffRcv = kOffP + kPBytes;                // the peer's partial scores [8 warps]
 constexpr int kOffRed = kOffRcv + kXBytes;              // row maxima / sums of both CTAs
 static_assert(kOffK % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "swizzle atom alignment");
 constexpr int kOffBar = kOffRed + kSlotFloats * 4;
@@ -320,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return mbar_test_wait(bar(kPFull), tp & 1);
       };
       auto issue_qk = [&]() {
+        MLA_TR(kTrQk, tq);
         const int st = tq % kStages;
         const int b = tq & 1;
         tc_fence_after();
@@ -336,12 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = smem_desc_sw64(kbase + 4 * kKBox + i * 32, 16, 512);
           umma_ss(dS, adesc, bdesc, idesc_qk, 1u);
         }
+        MLA_TR(kTrB, tq);
         umma_commit(bar(kSFull + b));
         if (wq.last()) umma_commit(bar(kQEmpty));
         wq.next(p);
         ++tq;
       };
       auto issue_pv = [&]() {
+        MLA_TR(kTrPv, tp);
         const int st = tp % kStages;
         tc_fence_after();
         const uint32_t vbase = sbase + kOffK + st * kStageBytes;
@@ -364,7 +368,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // time nothing is ready.
       long long idle_since = clock64();
       uint32_t polls = 0;
+#ifdef MLA_TRACE
+      uint32_t tdone = 0, pdone = 0;
+#endif
       while (wp.valid) {
+#ifdef MLA_TRACE
+        if (tdone < tq && mbar_test_wait(bar(kSFull + (tdone & 1)), (tdone >> 1) & 1)) {
+          MLA_TR(kTrC, tdone);
+          ++tdone;
+        }
+        if (pdone < tp && mbar_test_wait(bar(kPEmpty), pdone & 1)) {
+          MLA_TR(kTrD, pdone);
+          ++pdone;
+        }
+#endif
         if (tp < tq && pv_ready()) {
           issue_pv();
         } else if (wq.valid && tq < tp + 3 && qk_ready()) {
@@ -402,8 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int send_col = 32 * static_cast<int>(peer) + kOwnN * sub;   // S columns it sends to the peer
     // its P: tile 2c + sub (keys own_col ..), rows 32 q4 .. 32 q4 + 31 = one contiguous kilobyte
     const uint32_t p_piece = sbase + kOffP + (2 * crank + sub) * kPTile + q4 * 32 * 32;
-    uint8_t* stg_row = smem + kOffStg + sm * kXWarp + lane * kRowBytes;
-    const uint32_t stg_warp = sbase + kOffStg + sm * kXWarp;
     float* slots = reinterpret_cast<float*>(smem + kOffRed);  // [parity][source CTA][key quarter][row]
     // a quadrant whose 32 rows are all padding keeps the barrier protocol but skips the math;
     // its peer quadrant skips the same way
@@ -431,10 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // slot of parity x & 1 is written again only in exchange x + 2, which on either side follows
     // this thread's exchange x + 1 and so its reading of exchange x.
     uint32_t xc = 0;
-    // Lane 0's bulk copies alternate between the partial of a block (staging rows) and the P piece
-    // of a block; before rewriting either source, the copy that last read it must be done, and at
-    // most one copy of the other kind was committed after it.
-    int last_copy = 0;  // 0 none yet, 1 partial, 2 P piece
     auto xchg_post = [&](float v) {
       const int par = xc & 1;
       const uint32_t xb = bar(kXchg + 2 * q4 + par);
@@ -497,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool new_q = nx.valid && nx.chunk != wu.chunk;
       if (new_q && active) prefetch_q(nx.req);  // into L1 while the scores finish
       mbar_wait(bar(kSFull + b), (u >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      if (sm == 0 && lane == 0) MLA_TR(kTrSmS, u);
       __syncwarp();  // reconverge before the warp-collective tcgen05 ops
       tc_fence_after();
       if (new_q) {
@@ -514,37 +526,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t r[16];
       tmem_ld16(t_lane + kColS + 64 * b + send_col, r);
       tmem_wait_ld();
-      stamp(kTrA, u);
-      // the previous partial's copy out of the staging rows is done (a P copy committed since may
-      // still be reading)
-      if (lane == 0) {
-        if (last_copy == 2)
-          bulk_wait_read<1>();
-        else
-          bulk_wait_read_all();
-      }
-      __syncwarp();
-      stamp(kTrB, u);
       {
-        uint32_t w[kRowWords];  // 16 scores -> 12 words -> 3 chunks (48-byte rows: no bank conflicts)
+        uint32_t w[kRowWords];  // 16 scores -> 12 words -> three 16-byte stores into the peer's row
 #pragma unroll
         for (int g = 0; g < 4; ++g)
           pack24(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3], w[3 * g], w[3 * g + 1], w[3 * g + 2]);
+        // the peer's receive slot of this warp is free once the peer has combined block u - 1
+        if (lane == 0) mbar_wait<true>(bar(kXEmpty + sm), (u & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        __syncwarp();
+        stamp(kTrC, u);
+        const uint32_t dst = mapa(sbase + kOffRcv + sm * kXWarp + lane * kRowBytes, peer);
+        const uint32_t rb = mapa(bar(kXFull + sm), peer);
 #pragma unroll
         for (int j = 0; j < 3; ++j)
-          *reinterpret_cast<uint4*>(stg_row + 16 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          st_async_v4(dst + 16 * j, rb, __uint_as_float(w[4 * j]), __uint_as_float(w[4 * j + 1]),
+                      __uint_as_float(w[4 * j + 2]), __uint_as_float(w[4 * j + 3]));
       }
-      fence_proxy_async_smem();  // the bulk copy reads the staging through the async proxy
-      __syncwarp();
-      stamp(kTrC, u);
-      if (lane == 0) {
-        // the peer's receive slot of this warp is free once the peer has combined block u - 1
-        mbar_wait<true>(bar(kXEmpty + sm), (u & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        bulk_copy_to_peer(mapa(sbase + kOffRcv + sm * kXWarp, peer), stg_warp, kXWarp, mapa(bar(kXFull + sm), peer));
-        bulk_commit_group();
-      }
-      last_copy = 1;
-      __syncwarp();
       stamp(kTrSend, u);
     };
 
@@ -568,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float x[kOwnN];
       if (active) {
         mbar_wait<true>(bar(kXFull + sm), t & 1, abort_flag, err, kDevErrTimeout);
+        if (sm == 0 && lane == 0) MLA_TR(kTrSmX, t);
         __syncwarp();
         stamp(kTrSmX, t);
         uint32_t r[16];
@@ -632,6 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_cluster_relaxed_after(mapa(bar(kXEmpty + sm), peer), mx);
         }
         xchg_post(mx);
+        if (sm == 0 && lane == 0) MLA_TR(kTrSend, t);
         stamp(kTrQk, t);
       }
       if (wu.valid) {  // block t + 1's partial travels while block t's maximum does
@@ -639,6 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wu.next(p);
         ++u;
       }
+      if (sm == 0 && lane == 0) MLA_TR(kTrE, t);
       if (!active) {
         mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
@@ -655,6 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           xchg_wait(v);
           mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
         }
+        if (sm == 0 && lane == 0) MLA_TR(kTrSmC, t);
         stamp(kTrG, t);
         bool resc = false;
         float alpha = 1.f;
@@ -682,13 +683,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // P (this thread's 16 keys of the row), once this CTA's previous P.V has read P (so O also
         // holds every earlier block); then tell the peer it may copy its part of P here
         mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        if (sm == 0 && lane == 0) MLA_TR(kTrF, t);
+        stamp(kTrPv, t);
         if (lane == 0) {
           mbar_arrive_cluster_relaxed_after(mapa(bar(kPeerFree + sm), peer), 0.f);
-          // this piece's copy of the previous block is done (a partial's copy may follow it)
-          if (last_copy == 1)
-            bulk_wait_read<1>();
-          else
-            bulk_wait_read_all();
+          bulk_wait_read_all();  // this piece's copy of the previous block is done
         }
         __syncwarp();
         tc_fence_after();
@@ -700,13 +699,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();  // P is read by the tensor core and the bulk copy (async proxy)
         __syncwarp();
+        stamp(kTrA, t);
         if (lane == 0) {
           // the peer's P.V of the previous block has read its P too
           mbar_wait<true>(bar(kPeerFree + sm), t & 1, abort_flag, err, kDevErrTimeout);
+          if (sm == 0) MLA_TR(kTrG, t);
           bulk_copy_to_peer(mapa(p_piece, peer), p_piece, 1024, mapa(bar(kPFull), peer));
           bulk_commit_group();
         }
-        last_copy = 2;
         if (__any_sync(0xffffffffu, resc)) {
           // only blocks after the chunk's first can move an established reference, so O holds
           // the chunk's earlier blocks here; each warp of the quadrant rescales 128 of the 256 columns
@@ -730,6 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             mbar_arrive(bar(kPFull));
         }
+        if (sm == 0 && lane == 0) MLA_TR(kTrSmP, t);
         __syncwarp();
         stamp(kTrSmP, t);
       }
