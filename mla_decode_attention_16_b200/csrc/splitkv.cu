@@ -137,10 +137,6 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   }
 }
 
-// The value a 24-bit packed score stands for (pack24 keeps the top three bytes;
-// unpack24 puts back a half step): the same bits without unpacking.
-__device__ __forceinline__ float round24(uint32_t v) { return __uint_as_float((v & 0xFFFFFF00u) | 0x80u); }
-
 // Walks a partition's blocks in order: chunk after chunk (one chunk = the
 // partition's blocks of one request), block after block.
 struct Walk {
@@ -560,7 +556,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: this thread's keys' row sum relative to it
     for (uint32_t t = 0; wt.valid; ++t, wt.next(p)) {
       if (*abort_flag) break;
-      // ---- block t: own partial (rounded as sent) + the peer's, then release the score buffer
+      // ---- block t: own partial + the peer's, then release the score buffer.  Only this CTA
+      // computes the scores of its keys (the peer gets their P), so its own partial keeps full
+      // precision; the peer's arrives rounded to 24 bits.
       const int b = t & 1;
       float x[kOwnN];
       if (active) {
@@ -582,10 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float a0, a1, a2, a3;
           unpack24(wv[3 * g], wv[3 * g + 1], wv[3 * g + 2], a0, a1, a2, a3);
           const int c = 4 * g;
-          x[c] = round24(r[c]) + a0;
-          x[c + 1] = round24(r[c + 1]) + a1;
-          x[c + 2] = round24(r[c + 2]) + a2;
-          x[c + 3] = round24(r[c + 3]) + a3;
+          x[c] = __uint_as_float(r[c]) + a0;
+          x[c + 1] = __uint_as_float(r[c + 1]) + a1;
+          x[c + 2] = __uint_as_float(r[c + 2]) + a2;
+          x[c + 3] = __uint_as_float(r[c + 3]) + a3;
         }
         stamp(kTrE, t);
       }
