@@ -1,0 +1,76 @@
+"""Host-side logic of bench.py (no GPU): kernel choice, cost model, units, seeds, profile lookup."""
+
+import hashlib
+import importlib
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+bench = importlib.import_module("bench")
+from workloads import WORKLOADS, algorithmic_cost  # noqa: E402
+
+
+def test_kernel_choice_by_rows():
+    assert bench.kernel_of(1)[0] == "splitkv_narrow_kernel"
+    assert bench.kernel_of(32) == ("splitkv_narrow_kernel", "splitkv_narrow.cu")
+    assert bench.kernel_of(33) == ("splitkv_pair_kernel", "splitkv.cu")
+    assert bench.kernel_of(1024)[0] == "splitkv_pair_kernel"
+
+
+def test_cost_model_by_hand():
+    # two requests of 64 and 100 cached tokens, s_q 2, h_q 8: 16 rows, 164 tokens
+    c = algorithmic_cost([64, 100], 2, 8)
+    assert c["tokens"] == 164
+    assert c["flops"] == 2 * 16 * (576 + 512) * 164
+    assert c["kv_bytes"] == 576 * 2 * 164
+    assert c["bytes"] == 576 * 2 * 164 + 2 * 16 * (576 * 2 + 512 * 2 + 4)
+
+
+def test_units_and_throughput():
+    assert bench.unit_of("memory-bound") == "GB/s"
+    for name in ("compute-bound", "varlen-mtp", "long-fp16"):
+        assert bench.unit_of(name) == "TFLOPS", name
+    cost = {"bytes": 3e9, "flops": 5e12}
+    assert bench.throughput(cost, 0.5, "GB/s") == pytest.approx(6.0)
+    assert bench.throughput(cost, 0.5, "TFLOPS") == pytest.approx(10.0)
+
+
+def test_shard_seeds():
+    seeds = [bench.shard_seed(1001, r) for r in range(8)]
+    assert seeds[0] == 1001  # rank 0 runs the workload itself
+    assert len(set(seeds)) == 8
+
+
+def test_warmup_minimum_is_enforced():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2", "--steps", "1"])
+
+
+def test_profile_traffic_only_for_the_source_it_was_taken_from(tmp_path, monkeypatch):
+    csrc = tmp_path / "mla_decode_attention_16_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = csrc / "splitkv.cu"
+    src.write_bytes(b"// kernel source\n")
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    prof = tmp_path / "profiles" / "splitkv_pair_kernel_compute-bound.md"
+    prof.write_text(f"splitkv.cu sha256[:16]: {digest}\ntraffic_bytes_per_launch: 628559360.0\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profile_traffic("compute-bound", "splitkv_pair_kernel", "splitkv.cu") == 628559360.0
+    src.write_bytes(b"// kernel source, changed\n")  # counters no longer describe this kernel
+    assert bench.profile_traffic("compute-bound", "splitkv_pair_kernel", "splitkv.cu") is None
+    assert bench.profile_traffic("memory-bound", "splitkv_narrow_kernel", "splitkv_narrow.cu") is None
+
+
+def test_every_bench_workload_has_a_profile_summary():
+    for name in WORKLOADS:
+        if name == "tiny":
+            continue
+        kernel, _ = bench.kernel_of(WORKLOADS[name].rows)
+        if name in ("memory-bound", "compute-bound"):
+            assert os.path.exists(os.path.join(ROOT, "profiles", f"{kernel}_{name}.md")), name
