@@ -39,36 +39,26 @@ def _inputs():
     return [f for f in files if f.endswith((".cu", ".cuh", ".h"))]
 
 
-FLAGS_RECORD = LIB + ".flags"  # extra flags of the library in place (developer builds add some)
-
-
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
-    if os.path.exists(FLAGS_RECORD) and open(FLAGS_RECORD).read().strip():
-        return True  # the library in place is a developer build
     t = os.path.getmtime(LIB)
     return any(os.path.getmtime(f) > t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=(), out: str = LIB) -> str:
-    if not force and out == LIB and not extra_flags and not needs_build():
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not needs_build():
         return LIB
-    tmp = out + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC,
-           *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
+    tmp = LIB + ".tmp"
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *[os.path.join(CSRC, s) for s in SOURCES], "-o", tmp]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
-    os.replace(tmp, out)
-    if out == LIB:
-        with open(FLAGS_RECORD, "w") as f:
-            f.write(" ".join(extra_flags))
-    return out
+    os.replace(tmp, LIB)
+    return LIB
 
 
 if __name__ == "__main__":
-    flags = [a[len("--flag="):] for a in sys.argv[1:] if a.startswith("--flag=")]
-    print(build(force="--force" in sys.argv or bool(flags), verbose=True, extra_flags=flags))
+    print(build(force="--force" in sys.argv, verbose=True))

@@ -36,7 +36,6 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-long long* g_trace = nullptr;  // set only through mla_debug_set_trace in MLA_TRACE builds
 
 int ensure_encode() {
   if (g_encode) return MLA_OK;
@@ -206,7 +205,6 @@ int prepare(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int dtype
   p->block_table = nullptr;
   p->block_table_stride = 0;
   p->num_pages = 0;
-  p->trace = g_trace;
   return MLA_OK;
 }
 
@@ -262,13 +260,6 @@ int mla_last_cuda_error(void) { return g_last_cuda_error; }
 
 int mla_version(void) { return 100; }
 
-#ifdef MLA_TRACE
-// Developer builds only: device buffer of 6 x 1024 int64 clock stamps per block of CTA 0.
-int mla_debug_set_trace(long long* device_buffer) {
-  g_trace = device_buffer;
-  return MLA_OK;
-}
-#endif
 
 int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts) {
   if (!num_sm_parts || rows < 1) return MLA_ERR_INVALID_ARG;

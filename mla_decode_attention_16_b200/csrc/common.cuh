@@ -51,37 +51,6 @@ struct DecodeParams {
   int batch, s_q, h_q, rows, m_tiles, num_parts;
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
-  long long* trace;  // per-block timestamps of CTA 0 (only read by builds with MLA_TRACE)
 };
-
-// Developer trace events (stamped only by builds with MLA_TRACE).
-enum TraceEv { kTrProd = 0, kTrQk, kTrPv, kTrSmS, kTrSmX, kTrSmP, kTrSend, kTrSmC, kTrA, kTrB, kTrC, kTrD, kTrE, kTrF, kTrG, kTrH, kTrNum };
-constexpr int kTrMax = 1024;
-#ifdef MLA_TRACE
-// Per-block clock stamps of CTAs 0 and 1 into p.trace[cta][event][block].
-__device__ __forceinline__ void trace_stamp(const DecodeParams& p, int ev, uint32_t it) {
-  if (p.trace && blockIdx.x < 2 && it < kTrMax) p.trace[(blockIdx.x * kTrNum + ev) * kTrMax + it] = clock64();
-}
-#define MLA_TR(ev, it) trace_stamp(p, ev, it)
-// Global-timer stamps of every CTA (entry, after the dependency wait, end) after the per-block
-// area: p.trace[2*kTrNum*kTrMax + 3*cta + k].
-__device__ __forceinline__ void trace_cta(const DecodeParams& p, int k) {
-  if (p.trace && threadIdx.x == 0) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    p.trace[2 * kTrNum * kTrMax + 3 * blockIdx.x + k] = static_cast<long long>(t);
-    p.trace[2 * kTrNum * kTrMax + 3 * 4096 + 3 * blockIdx.x + k] = clock64();
-    if (k == 0) {
-      unsigned int smid;
-      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-      p.trace[2 * kTrNum * kTrMax + 6 * 4096 + blockIdx.x] = smid;
-    }
-  }
-}
-#define MLA_TR_CTA(k) trace_cta(p, k)
-#else
-#define MLA_TR_CTA(k) ((void)0)
-#define MLA_TR(ev, it) ((void)0)
-#endif
 
 }  // namespace mla

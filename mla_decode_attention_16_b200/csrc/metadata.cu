@@ -65,7 +65,7 @@ __device__ long long block_exclusive_scan(T* v, int n, long long* warp_tot) {
   return total;
 }
 
-__global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
+__global__ void __launch_bounds__(kThreads, 1) metadata_kernel(const int32_t* __restrict__ seqlens, int batch,
                                                             int num_parts, int32_t* __restrict__ meta,
                                                             int32_t* __restrict__ num_splits) {
   // smem: unit offset of each request (cum, int64) [batch + 1], then blocks / pieces per request (int32)
@@ -105,12 +105,8 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
   if (threadIdx.x == 0) num_splits[batch] = static_cast<int32_t>(total_pieces);
 
   // partition boundaries: unit x -> (last request with cum <= x, blocks of it before x), or (batch, 0)
-  auto locate = [&](long long x, int& r, int& k) {
-    if (share == 0 || x >= total) {
-      r = batch;
-      k = 0;
-      return;
-    }
+  auto locate = [&](long long x) -> int2 {
+    if (share == 0 || x >= total) return make_int2(batch, 0);
     int lo = 0, hi = batch - 1;  // largest r with s_cum[r] <= x (s_cum[0] = 0 <= x)
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -119,25 +115,17 @@ __global__ void __launch_bounds__(kThreads) metadata_kernel(const int32_t* __res
       else
         hi = mid - 1;
     }
-    r = lo;
     const long long off = x - s_cum[lo] - kFixedOverhead;
-    k = off > 0 ? static_cast<int>(off) : 0;
+    return make_int2(lo, off > 0 ? static_cast<int>(off) : 0);
   };
   for (int part = threadIdx.x; part < num_parts; part += kThreads) {
-    int br, bk, er, ek;
-    locate(static_cast<long long>(part) * share, br, bk);
-    locate(static_cast<long long>(part + 1) * share, er, ek);
+    const int2 b = locate(static_cast<long long>(part) * share);
+    const int2 e = locate(static_cast<long long>(part + 1) * share);
     int bsplit = 0;
-    if (bk > 0) bsplit = part - static_cast<int>((s_cum[br] + kFixedOverhead) / share);
-    int32_t* row = meta + part * kMetaInts;
-    row[0] = br;
-    row[1] = bk;
-    row[2] = er;
-    row[3] = ek;
-    row[4] = bsplit;
-    row[5] = 0;
-    row[6] = 0;
-    row[7] = 0;
+    if (b.y > 0) bsplit = part - static_cast<int>((s_cum[b.x] + kFixedOverhead) / share);
+    int4* row = reinterpret_cast<int4*>(meta + part * kMetaInts);
+    row[0] = make_int4(b.x, b.y, e.x, e.y);
+    row[1] = make_int4(bsplit, 0, 0, 0);
   }
 }
 

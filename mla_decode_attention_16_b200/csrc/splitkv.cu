@@ -178,24 +178,6 @@ struct Walk {
   __device__ __forceinline__ bool last() const { return blk == hi - 1; }
 };
 
-// Developer builds (MLA_TRACE): cycles a single-thread role spends in one kind of wait.
-struct WaitClock {
-#ifdef MLA_TRACE
-  long long acc[6] = {};
-  long long t0 = 0;
-  __device__ __forceinline__ void start() { t0 = clock64(); }
-  __device__ __forceinline__ void stop(int slot) { acc[slot] += clock64() - t0; }
-  __device__ __forceinline__ void dump(const DecodeParams& p, int column) const {
-    if (p.trace && blockIdx.x < 2)
-      for (int e = 0; e < 6; ++e) p.trace[(blockIdx.x * kTrNum + e) * kTrMax + column] = acc[e];
-  }
-#else
-  __device__ __forceinline__ void start() {}
-  __device__ __forceinline__ void stop(int) {}
-  __device__ __forceinline__ void dump(const DecodeParams&, int) const {}
-#endif
-};
-
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_pair_kernel(const void* __restrict__ qptr, const __grid_constant__ CUtensorMap qrmap,
@@ -210,7 +192,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  MLA_TR_CTA(0);
   const uint32_t crank = cluster_ctarank();
   const uint32_t peer = crank ^ 1u;
   const int pair = blockIdx.x >> 1;
@@ -245,7 +226,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // scheduler): everything above overlapped it; nothing it wrote is read before this wait
   pdl_wait_primary();
   if (threadIdx.x == 0) pdl_launch_dependents();
-  MLA_TR_CTA(1);
 
   const int* meta = p.meta + part * kMetaInts;
   const int R = p.rows;
@@ -257,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t evict_first = policy_evict_first();
       Walk w;
       w.init(p, meta);
-      WaitClock wc;
       auto page_of = [&](const Walk& x) {
         return x.valid ? p.block_table[static_cast<int64_t>(x.req) * p.block_table_stride + x.blk] : 0;
       };
@@ -268,9 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         Walk nx = w;
         nx.next(p);
         page_next = page_of(nx);  // the next block's page index is read while this stage frees up
-        wc.start();
         mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        wc.stop(0);
         if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
           atomicOr(err, kDevErrPage);
           atomicCAS(err + 1, 0, page == 0 ? -1 : page);
@@ -283,15 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_hint(dst + 4 * kKBox, &krmap, bar(kKvFull + st), 512 + 32 * crank, 0, page, evict_first);
         if (w.first()) {
           // the chunk's Q columns 512 + 32c .., once the previous chunk's last Q.K^T has read the old ones
-          wc.start();
           mbar_wait(bar(kQEmpty), (w.chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-          wc.stop(1);
           mbar_arrive_expect_tx(bar(kQrFull), kQrBox);
           tma_load_2d(sbase + kOffQR, &qrmap, bar(kQrFull), 512 + 32 * crank, w.req * R + mtile * kTileRows);
         }
         w = nx;
       }
-      wc.dump(p, 9);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -302,7 +276,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       wq.init(p, meta);
       wp = wq;
       uint32_t tq = 0, tp = 0;
-      WaitClock wc;
       // Inputs of the next Q.K^T (chunk's Q, the page, a free score buffer) / the next P.V (P, and
       // for a chunk's first block the epilogue having read O) are complete.  Each barrier phase
       // tested here cannot run a full phase ahead: its producer waits on this thread's earlier work.
@@ -317,7 +290,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         return mbar_test_wait(bar(kPFull), tp & 1);
       };
       auto issue_qk = [&]() {
-        MLA_TR(kTrQk, tq);
         const int st = tq % kStages;
         const int b = tq & 1;
         tc_fence_after();
@@ -334,14 +306,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = smem_desc_sw64(kbase + 4 * kKBox + i * 32, 16, 512);
           umma_ss(dS, adesc, bdesc, idesc_qk, 1u);
         }
-        MLA_TR(kTrB, tq);
         umma_commit(bar(kSFull + b));
         if (wq.last()) umma_commit(bar(kQEmpty));
         wq.next(p);
         ++tq;
       };
       auto issue_pv = [&]() {
-        MLA_TR(kTrPv, tp);
         const int st = tp % kStages;
         tc_fence_after();
         const uint32_t vbase = sbase + kOffK + st * kStageBytes;
@@ -364,20 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // time nothing is ready.
       long long idle_since = clock64();
       uint32_t polls = 0;
-#ifdef MLA_TRACE
-      uint32_t tdone = 0, pdone = 0;
-#endif
       while (wp.valid) {
-#ifdef MLA_TRACE
-        if (tdone < tq && mbar_test_wait(bar(kSFull + (tdone & 1)), (tdone >> 1) & 1)) {
-          MLA_TR(kTrC, tdone);
-          ++tdone;
-        }
-        if (pdone < tp && mbar_test_wait(bar(kPEmpty), pdone & 1)) {
-          MLA_TR(kTrD, pdone);
-          ++pdone;
-        }
-#endif
         if (tp < tq && pv_ready()) {
           issue_pv();
         } else if (wq.valid && tq < tp + 3 && qk_ready()) {
@@ -398,7 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(bar(kDrain));
       mbar_wait_drain(bar(kDrain), 0);
-      wc.dump(p, 8);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ Q to TMEM, exchange, softmax, correction, epilogue
@@ -420,19 +376,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // its peer quadrant skips the same way
     const bool active = mtile * kTileRows + q4 * 32 < R;
     const int active_quadrants = min(4, (R - mtile * kTileRows + 31) / 32);
-#ifdef MLA_TRACE
-    // developer builds: cycles spent per section, summed over the blocks
-    long long tr_acc[kTrNum] = {};
-    long long tr_prev = clock64();
-#endif
-    auto stamp = [&](int ev, uint32_t) {
-#ifdef MLA_TRACE
-      const long long now = clock64();
-      tr_acc[ev] += now - tr_prev;
-      tr_prev = now;
-#endif
-      (void)ev;
-    };
 
     // The row's four values of one kind (its block maximum, its row sum), one per thread of the
     // row in either CTA: post puts this thread's into this CTA's slot and (a 4-byte distributed
@@ -504,7 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool new_q = nx.valid && nx.chunk != wu.chunk;
       if (new_q && active) prefetch_q(nx.req);  // into L1 while the scores finish
       mbar_wait(bar(kSFull + b), (u >> 1) & 1, abort_flag, err, kDevErrTimeout);
-      if (sm == 0 && lane == 0) MLA_TR(kTrSmS, u);
       __syncwarp();  // reconverge before the warp-collective tcgen05 ops
       tc_fence_after();
       if (new_q) {
@@ -517,7 +459,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kQtFull));
       }
-      stamp(kTrSmS, u);
       if (!active) return;
       uint32_t r[16];
       tmem_ld16(t_lane + kColS + 64 * b + send_col, r);
@@ -530,7 +471,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the peer's receive slot of this warp is free once the peer has combined block u - 1
         if (lane == 0) mbar_wait<true>(bar(kXEmpty + sm), (u & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
-        stamp(kTrC, u);
         const uint32_t dst = mapa(sbase + kOffRcv + sm * kXWarp + lane * kRowBytes, peer);
         const uint32_t rb = mapa(bar(kXFull + sm), peer);
 #pragma unroll
@@ -538,7 +478,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_async_v4(dst + 16 * j, rb, __uint_as_float(w[4 * j]), __uint_as_float(w[4 * j + 1]),
                       __uint_as_float(w[4 * j + 2]), __uint_as_float(w[4 * j + 3]));
       }
-      stamp(kTrSend, u);
     };
 
     Walk wu, wt;
@@ -563,13 +502,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float x[kOwnN];
       if (active) {
         mbar_wait<true>(bar(kXFull + sm), t & 1, abort_flag, err, kDevErrTimeout);
-        if (sm == 0 && lane == 0) MLA_TR(kTrSmX, t);
         __syncwarp();
-        stamp(kTrSmX, t);
         uint32_t r[16];
         tmem_ld16(t_lane + kColS + 64 * b + own_col, r);
         tmem_wait_ld();
-        stamp(kTrD, t);
         const uint8_t* rcv_row = smem + kOffRcv + sm * kXWarp + lane * kRowBytes;
         const uint4 c0 = *reinterpret_cast<const uint4*>(rcv_row);
         const uint4 c1 = *reinterpret_cast<const uint4*>(rcv_row + 16);
@@ -585,12 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           x[c + 2] = __uint_as_float(r[c + 2]) + a2;
           x[c + 3] = __uint_as_float(r[c + 3]) + a3;
         }
-        stamp(kTrE, t);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kSEmpty + b));  // Q.K^T of block t + 2 may overwrite the scores
-      stamp(kTrSmC, t);
 
       if (wt.first()) {
         m = -INFINITY;
@@ -618,7 +552,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mx = fmaxf(mx, x[c]);
           }
         }
-        stamp(kTrF, t);
         __syncwarp();
         if (lane == 0) {
           // every lane's mx was computed from every word it read from the receive slot, so those
@@ -628,15 +561,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_cluster_relaxed_after(mapa(bar(kXEmpty + sm), peer), mx);
         }
         xchg_post(mx);
-        if (sm == 0 && lane == 0) MLA_TR(kTrSend, t);
-        stamp(kTrQk, t);
       }
       if (wu.valid) {  // block t + 1's partial travels while block t's maximum does
         send_partial(u, wu);
         wu.next(p);
         ++u;
       }
-      if (sm == 0 && lane == 0) MLA_TR(kTrE, t);
       if (!active) {
         mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         __syncwarp();
@@ -653,8 +583,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           xchg_wait(v);
           mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
         }
-        if (sm == 0 && lane == 0) MLA_TR(kTrSmC, t);
-        stamp(kTrG, t);
         bool resc = false;
         float alpha = 1.f;
         if (mx > m + kRescaleThreshold) {  // also true when m is still -inf and a key is visible
@@ -676,13 +604,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c2] = pack2<kBF16>(p0, p1);
         }
         l = l * alpha + (s0 + s1);
-        stamp(kTrH, t);
 
         // P (this thread's 16 keys of the row), once this CTA's previous P.V has read P (so O also
         // holds every earlier block); then tell the peer it may copy its part of P here
         mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        if (sm == 0 && lane == 0) MLA_TR(kTrF, t);
-        stamp(kTrPv, t);
         if (lane == 0) {
           mbar_arrive_cluster_relaxed_after(mapa(bar(kPeerFree + sm), peer), 0.f);
           bulk_wait_read_all();  // this piece's copy of the previous block is done
@@ -697,11 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();  // P is read by the tensor core and the bulk copy (async proxy)
         __syncwarp();
-        stamp(kTrA, t);
         if (lane == 0) {
           // the peer's P.V of the previous block has read its P too
           mbar_wait<true>(bar(kPeerFree + sm), t & 1, abort_flag, err, kDevErrTimeout);
-          if (sm == 0) MLA_TR(kTrG, t);
           bulk_copy_to_peer(mapa(p_piece, peer), p_piece, 1024, mapa(bar(kPFull), peer));
           bulk_commit_group();
         }
@@ -728,9 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             mbar_arrive(bar(kPFull));
         }
-        if (sm == 0 && lane == 0) MLA_TR(kTrSmP, t);
         __syncwarp();
-        stamp(kTrSmP, t);
       }
 
       if (!wt.last()) continue;
@@ -792,17 +713,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kOEmpty));
-      stamp(kTrProd, t);  // epilogue
     }
     if (lane == 0) bulk_wait_read_all();
-#ifdef MLA_TRACE
-    if (lane == 0 && p.trace && blockIdx.x < 2)
-      for (int e = 0; e < kTrNum; ++e) p.trace[(blockIdx.x * kTrNum + e) * kTrMax + sm] = tr_acc[e];
-#endif
   }
 
   // ------------------------------------------------------------ teardown
-  MLA_TR_CTA(2);
   __syncwarp();  // lanes of the producer / MMA warps rejoin their elected lane
   tc_fence_before();
   __syncthreads();

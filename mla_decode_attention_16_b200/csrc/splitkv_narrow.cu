@@ -141,7 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  MLA_TR_CTA(0);
   const int part = blockIdx.x;
 
   if (threadIdx.x == 0) {
@@ -165,7 +164,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   // scheduler): the prologue above overlapped it; nothing it wrote is read before this wait
   pdl_wait_primary();
   if (threadIdx.x == 0) pdl_launch_dependents();
-  MLA_TR_CTA(1);
 
   const int* meta = p.meta + part * kMetaInts;
   const int br = meta[0], bk = meta[1], er = meta[2], ek = meta[3], bs = meta[4];
@@ -193,7 +191,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicCAS(err + 1, 0, page == 0 ? -1 : page);
             page = 0;
           }
-          MLA_TR(kTrProd, it);
           mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
           for (int i = 0; i < kBoxes; ++i)
             tma_load_3d_hint(sbase + Lay::kOffK + st * kStageBytes + i * kKBox, &kmap, bar(kKvFull + st), 64 * i,
@@ -214,7 +211,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (jjp == 0) mbar_wait(bar(kOEmpty + ob), ((chunk / kOBufs) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
         mbar_wait(bar(kPFull + b), (itp >> 1) & 1, abort_flag, err, kDevErrTimeout);
         tc_fence_after();
-        MLA_TR(kTrPv, itp);
         const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
         const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
         const uint32_t dcol = tmem + Lay::kColO + ob * 128;
@@ -247,7 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, abort_flag, err, kDevErrTimeout);
           mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, abort_flag, err, kDevErrTimeout);
           tc_fence_after();
-          MLA_TR(kTrQk, itc);
           const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
 #pragma unroll 1
           for (int i = 0; i < kBoxes; ++i) {
@@ -294,7 +289,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kSFull), itc & 1, abort_flag, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
-          if (lane == 0) MLA_TR(kTrSmS, itc);
           float x[64];
           {
             uint32_t r0[32], r1[32];
@@ -352,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                   make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
           }
           fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
-          if (lane == 0) MLA_TR(kTrSmP, itc);
         }
         named_bar_sync(1, 128);
         if (s_flag[b] && jj > 0) {
@@ -496,7 +489,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  MLA_TR_CTA(2);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);

@@ -28,7 +28,7 @@ kernel reaches up to rounding order):
   cached tokens per request, ``causal`` masks future tokens, and the
   log-sum-exp of the scaled scores is returned beside the output.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * lse is the natural log of sum_j exp(scale * q.k_j) (scaled-score units).
 * causal with s_q > 1 is aligned bottom-right: query position s (0-based) of

@@ -15,8 +15,7 @@ Sources:
   blocks to the SMs so variable-length batches stay balanced.
 * same walk-through, section 项目主要功能: a block is one 64-token page.
 
-Reading (the pages give the share formula, not the assignment; listed in
-DESIGN.md):
+Reading taken here (the pages give the share formula, not the assignment):
 * n_r = ceil(L_r / 64) blocks per request; F = 3 units of fixed overhead per
   request that has blocks.  The pages name fixed_overhead_num_blocks without a
   value; F is a tuning constant of the scheduler (every F gives a valid
