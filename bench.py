@@ -2,10 +2,13 @@
 
 A step is one pass of the whole hot path over one batch: the tile scheduler
 (mla_get_metadata) followed by the decode forward (split-KV kernel + combine
-kernel), inputs resident in HBM.  The default workload is the memory-bound
-decode batch (64 requests x 4096 cached tokens, h_q 16, s_q 1, bf16); pick
-another with --workload.  Throughput uses the pages' cost model:
-bytes = 576*2*sum(L) + q + out + lse, FLOPs = 2*h_q*s_q*(576+512)*sum(L).
+kernel), inputs resident in HBM.  The headline workload is the memory-bound
+decode batch (64 requests x 4096 cached tokens, h_q 16, s_q 1, bf16); a
+default run adds, under "per_workload", the same measurements for the three
+workloads with h_q * s_q >= 128 (compute-bound, varlen-mtp, long-fp16; at most
+--companion-steps timed steps each).  Pick one workload with --workload.
+Throughput uses the pages' cost model: bytes = 576*2*sum(L) + q + out + lse,
+FLOPs = 2*h_q*s_q*(576+512)*sum(L).
 
 Timing: W warm-up steps, then exactly K steps between CUDA events on the
 launching stream, with a barrier and a synchronize on both sides; two resident
@@ -248,9 +251,7 @@ def workload_config(name: str, world: int):
 
 
 # ----------------------------------------------------------------------------- GPU leg
-def run_gpu(args, name: str):
-    import mla_decode_attention_16_b200 as mla
-
+def init_dist():
     world, rank, local = dist_env()
     if world > 1:
         import datetime
@@ -262,18 +263,25 @@ def run_gpu(args, name: str):
                                 device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
+    return world, rank, torch.device("cuda", torch.cuda.current_device())
+
+
+def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, cpu_seconds: float):
+    """Device throughput, split-KV kernel time, end-to-end throughput (and, on rank 0 of a 1-GPU run
+    with cpu_seconds > 0, the CPU oracle's) of one workload.  Every rank makes the same collective
+    calls in the same order; rank 0 gets the result dict, the others None."""
+    import mla_decode_attention_16_b200 as mla
+
     unit = unit_of(name)
     w = WORKLOADS[name]
-
-    inp = make_workload(name) if rank == 0 else None
-    if rank != 0:
+    if rank == 0:
+        inp = make_workload(name)
+    else:
         import workloads as wl
-        g_inp = wl.make_case  # rank shards differ only by seed; same shapes and length law
-        g = torch.Generator().manual_seed(shard_seed(w.seed, rank))
+        g = torch.Generator().manual_seed(shard_seed(w.seed, rank))  # same shapes and length law
         lens = wl.draw_seqlens(w, g)
-        inp = g_inp(w.batch, w.s_q, w.h_q, lens, dtype=w.dtype, std=w.std, causal=w.causal,
-                    seed=shard_seed(w.seed, rank) + 1)
+        inp = wl.make_case(w.batch, w.s_q, w.h_q, lens, dtype=w.dtype, std=w.std, causal=w.causal,
+                           seed=shard_seed(w.seed, rank) + 1)
     lens = [int(x) for x in inp.cache_seqlens.tolist()]
     cost = algorithmic_cost(lens, inp.s_q, inp.h_q)
 
@@ -303,32 +311,32 @@ def run_gpu(args, name: str):
         torch.cuda.synchronize(dev)
 
     # ---- warm-up
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i)
     barrier()
     flags = mla.mla_read_device_status(ws, stream)
     if flags[0] != 0:
-        raise RuntimeError(f"device error flags {flags}")
+        raise RuntimeError(f"{name}: device error flags {flags}")
 
     # ---- timed region (device throughput, inputs resident)
     clocks = ClockSampler(dev.index)
-    est_s = 2e-4 * args.steps
+    est_s = 2e-4 * steps
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     clocks.start()
     torch.cuda._sleep(int(min(est_s, 0.5) * 1.0e9))  # head start so the host enqueues ahead of the GPU
     ev0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         step(i)
     ev1.record(stream)
     barrier()
     clocks.stop()
     elapsed = ev0.elapsed_time(ev1) / 1000.0
     elapsed_max = reduce_max(elapsed, dev)
-    value = throughput(cost, elapsed_max / args.steps, unit) * world
+    value = throughput(cost, elapsed_max / steps, unit) * world
 
     # ---- split-KV kernel alone, CUDA events per launch on the launching stream (roofline)
-    n_prof = max(3, min(args.steps, 200))
+    n_prof = max(3, min(steps, 200))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_prof)]
     mla.mla_get_metadata(sl, rows, parts, meta, ns, stream=stream)
     barrier()
@@ -339,7 +347,7 @@ def run_gpu(args, name: str):
                             stream=stream)
         z.record(stream)
     barrier()
-    kern_s = statistics.mean(a.elapsed_time(z) for a, z in evs) / 1000.0
+    kern_s = reduce_max(statistics.mean(a.elapsed_time(z) for a, z in evs) / 1000.0, dev)
 
     # ---- end to end through the public API with pinned host buffers.  A serving loop pipelines
     # steps: step i's inputs go host -> device on one stream while step i-1 computes on another
@@ -353,7 +361,7 @@ def run_gpu(args, name: str):
     lse_h = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
     h2d = q_h.numel() * q_h.element_size() + bt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h[0].numel() * out_h[0].element_size() + lse_h[0].numel() * 4
-    n_e2e = max(3, min(args.steps, 200))
+    n_e2e = max(3, min(steps, 200))
     q_d = [torch.empty_like(q) for _ in range(2)]
     bt_d = [torch.empty_like(bt) for _ in range(2)]
     sl_d = [torch.empty_like(sl) for _ in range(2)]
@@ -399,12 +407,12 @@ def run_gpu(args, name: str):
     barrier()
     e2e_s = reduce_max(e0.elapsed_time(e1) / 1000.0 / n_e2e, dev)
     e2e_value = throughput(cost, e2e_s, unit) * world
-
+    flags = mla.mla_read_device_status(ws, stream)
+    if flags[0] != 0:
+        raise RuntimeError(f"{name}: device error flags {flags}")
+    del caches, q_d, out_d
     if rank != 0:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
-        return 0
+        return None
 
     peaks, peak_src = load_peaks()
     if unit == "GB/s":
@@ -415,28 +423,53 @@ def run_gpu(args, name: str):
         achieved = cost["flops"] / kern_s / 1e12
         peak = float(peaks["bf16_tflops"])  # fp16 dense tensor rate equals bf16 on this part
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
-    kname, ksrc = kernel_of(inp.s_q * inp.h_q)
+    kname, ksrc = kernel_of(rows)
     roof["traffic"] = profile_traffic(name, kname, ksrc)
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["kernel"] = kname
     roof["kernel_us"] = kern_s * 1e6
     roof["algorithmic_per_launch"] = cost["bytes"] if unit == "GB/s" else cost["flops"]
-
-    line = {
-        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000.0 * elapsed_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if q.dtype == torch.bfloat16 else "fp16",
-        "data": "synthetic", "config": workload_config(name, world),
-        "tflops": cost["flops"] / (elapsed_max / args.steps) / 1e12 * world,
-        "gbps": cost["bytes"] / (elapsed_max / args.steps) / 1e9 * world,
+    res = {
+        "value": value, "unit": unit, "steps": steps, "warmup": warmup,
+        "ms_per_step": 1000.0 * elapsed_max / steps,
+        "dtype": "bf16" if q.dtype == torch.bfloat16 else "fp16",
+        "config": workload_config(name, world),
+        "tflops": cost["flops"] / (elapsed_max / steps) / 1e12 * world,
+        "gbps": cost["bytes"] / (elapsed_max / steps) / 1e9 * world,
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 3 * steps,
         "clocks": clocks.summary(),
     }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inp, name, unit, args.cpu_seconds)
-    print(json.dumps(line), flush=True)
+    if world == 1 and cpu_seconds > 0:
+        res["cpu_baseline"] = cpu_baseline(inp, name, unit, cpu_seconds)
+    return res
+
+
+# workloads whose numbers join the headline line of a default run (the pages' h_q * s_q >= 128 configs)
+COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16"]
+
+
+def run_gpu(args, name: str, companions=()):
+    world, rank, dev = init_dist()
+    cpu_s = 0.0 if args.no_cpu_baseline else args.cpu_seconds
+    head = measure_gpu(name, args.steps, args.warmup, world, rank, dev, cpu_s)
+    extra = {}
+    for other in companions:
+        torch.cuda.empty_cache()
+        extra[other] = measure_gpu(other, min(args.steps, args.companion_steps), args.warmup, world, rank, dev,
+                                   0.0 if args.no_cpu_baseline else args.companion_cpu_seconds)
+    if rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
+                "data": "synthetic"}
+        for k in ("config", "tflops", "gbps", "roofline", "e2e", "gpu_launches", "clocks", "cpu_baseline"):
+            if k in head:
+                line[k] = head[k]
+        if extra:
+            line["per_workload"] = extra
+        print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -452,15 +485,31 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + ["all"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--companion-steps", type=int, default=200,
+                    help="timed steps of each h_q*s_q >= 128 workload added to a default run's line")
+    ap.add_argument("--companion-cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="a default run measures only the headline workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    names = [n for n in WORKLOADS if n != "tiny"] if args.workload == "all" else [args.workload]
-    for name in names:
-        rc = run_reference(args, name) if args.impl == "reference" else run_gpu(args, name)
-        if rc:
-            return rc
-    return 0
+    if args.impl == "reference":
+        names = [n for n in WORKLOADS if n != "tiny"] if args.workload == "all" else [args.workload]
+        for name in names:
+            rc = run_reference(args, name)
+            if rc:
+                return rc
+        return 0
+    if args.workload == "all":
+        for name in [n for n in WORKLOADS if n != "tiny"]:
+            rc = run_gpu(args, name)
+            if rc:
+                return rc
+        return 0
+    given = argv if argv is not None else sys.argv[1:]
+    default_run = not any(a.startswith("--workload") for a in given)
+    companions = COMPANIONS if default_run and not args.headline_only else ()
+    return run_gpu(args, args.workload, companions)
 
 
 if __name__ == "__main__":

@@ -27,7 +27,8 @@
  *    these paths and keeps only a per-device cache of SM counts and kernel
  *    attributes.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
- *    enqueue work; none synchronises except mla_read_device_status.
+ *    enqueue work; none synchronises except mla_read_device_status and
+ *    mla_static_ws_read_device_status.
  *  - Return value: MLA_OK (0) or an mla_status code.  Arguments are checked on
  *    the host before anything is enqueued; a failed check enqueues nothing.
  *    A failed CUDA launch returns MLA_ERR_CUDA and mla_last_cuda_error() gives
@@ -56,6 +57,7 @@ extern "C" {
 
 #define MLA_DEVERR_TIMEOUT 1
 #define MLA_DEVERR_PAGE_INDEX 2
+#define MLA_DEVERR_APPEND_POS 4 /* a request had fewer cached tokens than new ones */
 
 typedef enum {
   MLA_OK = 0,
@@ -154,6 +156,43 @@ int mla_decode_fwd(const void* q, const void* kcache, int64_t num_pages, const i
                    void* out, float* lse, void* stream);
 
 /*
+ * Append of the s_q new tokens' latent rows to the paged cache, the step that
+ * precedes the decode ("FlashMLA: 高性能GPU注意力机制计算库", section 项目主要功能:
+ * paged cache of 64-token blocks).
+ *   kv_new            device [batch, s_q, 576], dtype, contiguous, 16-B aligned:
+ *                     the new tokens' rows (key = all 576 values, value = the
+ *                     first 512)
+ *   kcache            device [num_pages, 64, 1, 576], written in place
+ *   cache_seqlens     device int32 [batch]: L_b, counting the new tokens, so
+ *                     new token s goes to position L_b - s_q + s, i.e. page
+ *                     block_table[b, (L_b - s_q + s) / 64], slot (.. % 64)
+ *   workspace         device, >= 256 bytes, 256-B aligned: its error word gets
+ *                     MLA_DEVERR_PAGE_INDEX (page outside [0, num_pages); the
+ *                     row is skipped) or MLA_DEVERR_APPEND_POS (L_b < s_q; the
+ *                     rows without a position are skipped)
+ * Every other argument as in mla_decode_fwd.  Rows of different requests must
+ * not share a slot.  Enqueues one kernel as a programmatic dependent launch: it
+ * sets up while the previous kernel in the stream finishes and writes nothing
+ * before that kernel has completed.
+ */
+int mla_append_kv(const void* kv_new, void* kcache, int64_t num_pages, const int32_t* block_table,
+                  int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The decode step fused with the append: mla_append_kv, then the split-KV and
+ * combine kernels of mla_decode_fwd, each a programmatic dependent launch of
+ * the one before on `stream` (the split-KV kernel reads pages only after the
+ * append has completed).  Arguments as in mla_decode_fwd and mla_append_kv;
+ * kcache is written.  Checks run before anything is enqueued.
+ */
+int mla_decode_fwd_append(const void* q, const void* kv_new, void* kcache, int64_t num_pages,
+                          const int32_t* block_table, int64_t block_table_stride, const int32_t* cache_seqlens,
+                          int batch, int s_q, int h_q, int dtype, float softmax_scale, int causal,
+                          const int32_t* tile_sched_metadata, const int32_t* num_splits, int num_sm_parts,
+                          void* workspace, size_t workspace_bytes, void* out, float* lse, void* stream);
+
+/*
  * The two stages of mla_decode_fwd, exposed for timing and testing; same
  * arguments and checks.  mla_splitkv_fwd writes out/lse of every request that
  * was not cut and the partials of the others; mla_combine_fwd merges the
@@ -188,13 +227,39 @@ int mla_combine_fwd(const int32_t* cache_seqlens, int batch, int s_q, int h_q, i
  * scratch array, which keeps the previous call's contents (its error header is
  * cleared at the start of every call), so calls that may overlap on the GPU --
  * on different streams, or on the same device from different threads without
- * ordering -- race and must not be issued.
+ * ordering -- race and must not be issued.  The cached address assumes the
+ * device is not reset (cudaDeviceReset) while the library stays loaded.
+ * Device-side errors of a call go to the scratch's error header:
+ * mla_static_ws_read_device_status reads them until the next call clears it.
  */
 int mla_decode_fwd_static_ws(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
                              int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q,
                              int h_q, int dtype, float softmax_scale, int causal,
                              const int32_t* tile_sched_metadata, const int32_t* num_splits, int num_sm_parts,
                              void* out, float* lse, void* stream);
+
+/*
+ * Companion of mla_decode_fwd_static_ws (no counterpart in the pages either):
+ * copies the error word (MLA_DEVERR_* bits) and the first offending page index
+ * of the built-in scratch on the current device to host `flags[2]`, i.e. the
+ * device status of the last mla_decode_fwd_static_ws call on that device;
+ * synchronises `stream`.  Does not clear them.
+ */
+int mla_static_ws_read_device_status(void* stream, int32_t* flags);
+
+/*
+ * Test hook for the kernels' bounded waits (no counterpart in the pages; never
+ * needed in production).  With enable = 1, every split-KV launch that follows
+ * (from any thread of the process) leaves out one software arrival -- the
+ * "query rows are in tensor memory" signal of the partition's first chunk -- so
+ * the pipeline stage waiting for it gives up after its wait limit, records
+ * MLA_DEVERR_TIMEOUT in the workspace's error word and the kernel returns
+ * (its outputs are then undefined).  wait_cycles > 0 sets the limit of every
+ * pipeline wait in SM clock cycles for those launches (0 = the default of about
+ * 2 s).  mla_test_withhold_q_ready(0, 0) restores normal operation.
+ * Returns MLA_ERR_INVALID_ARG for enable outside {0, 1} or wait_cycles < 0.
+ */
+int mla_test_withhold_q_ready(int enable, long long wait_cycles);
 
 /*
  * Copy the workspace's error word (MLA_DEVERR_* bits) and the first offending

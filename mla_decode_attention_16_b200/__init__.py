@@ -35,6 +35,8 @@ __all__ = [
     "mla_decode_fwd",
     "mla_splitkv_fwd",
     "mla_combine_fwd",
+    "mla_append_kv",
+    "mla_decode_fwd_append",
     "mla_read_device_status",
     "HEAD_DIM_K",
     "HEAD_DIM_V",
@@ -74,8 +76,12 @@ def _load() -> ctypes.CDLL:
     L.mla_splitkv_fwd.argtypes = fwd
     L.mla_combine_fwd.argtypes = [vp, c_int, c_int, c_int, c_int, vp, c_int, vp, c_sz, vp, vp, vp]
     L.mla_read_device_status.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int32)]
+    L.mla_append_kv.argtypes = [vp, vp, c_i64, vp, c_i64, vp, c_int, c_int, c_int, vp, c_sz, vp]
+    L.mla_decode_fwd_append.argtypes = [vp, vp, vp, c_i64, vp, c_i64, vp, c_int, c_int, c_int, c_int, c_f, c_int,
+                                        vp, vp, c_int, vp, c_sz, vp, vp, vp]
     for name in ("mla_get_num_sm_parts", "mla_get_workspace_size", "mla_get_metadata", "mla_decode_fwd",
-                 "mla_splitkv_fwd", "mla_combine_fwd", "mla_read_device_status"):
+                 "mla_splitkv_fwd", "mla_combine_fwd", "mla_read_device_status", "mla_append_kv",
+                 "mla_decode_fwd_append"):
         getattr(L, name).restype = c_int
     return L
 
@@ -221,6 +227,42 @@ def mla_combine_fwd(cache_seqlens, s_q, h_q, dtype, num_splits, num_sm_parts, wo
     _check(lib.mla_combine_fwd(_ptr(cache_seqlens), b, int(s_q), int(h_q), _DTYPES[dtype], _ptr(num_splits),
                                int(num_sm_parts), _ptr(workspace), workspace.numel(), _ptr(out), _ptr(lse),
                                _stream(stream, cache_seqlens.device)), "mla_combine_fwd")
+    return out, lse
+
+
+def _check_kv_new(kv_new, kcache, block_table):
+    _need(kv_new, "kv_new", kcache.dtype, 3)
+    if kv_new.shape[0] != block_table.shape[0] or kv_new.shape[2] != HEAD_DIM_K:
+        raise MlaError(f"kv_new must be [batch, s_q, {HEAD_DIM_K}], got {tuple(kv_new.shape)}")
+
+
+def mla_append_kv(kv_new, kcache, block_table, cache_seqlens, workspace, stream=None):
+    """Write kv_new [b, s_q, 576] into the cache at positions L_b - s_q + s (in place); see
+    include/mla_decode.h.  Returns kcache."""
+    _need(kcache, "kcache", dim=4)
+    if kcache.dtype not in _DTYPES:
+        raise MlaError(f"kcache must be bf16 or fp16, got {kcache.dtype}")
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8, 1)
+    _check_kv_new(kv_new, kcache, block_table)
+    b, s_q, _ = kv_new.shape
+    _check(lib.mla_append_kv(_ptr(kv_new), _ptr(kcache), kcache.shape[0], _ptr(block_table), block_table.stride(0),
+                             _ptr(cache_seqlens), b, s_q, _DTYPES[kcache.dtype], _ptr(workspace), workspace.numel(),
+                             _stream(stream, kcache.device)), "mla_append_kv")
+    return kcache
+
+
+def mla_decode_fwd_append(q, kv_new, kcache, block_table, cache_seqlens, softmax_scale, causal,
+                          tile_sched_metadata, num_splits, workspace=None, out=None, lse=None, stream=None):
+    """The decode step fused with the append of kv_new [b, s_q, 576] (kcache is written first);
+    returns out [b, s_q, h_q, 512] and lse [b, h_q, s_q]."""
+    args, out, lse = _fwd_args(q, kcache, block_table, cache_seqlens, softmax_scale, causal, tile_sched_metadata,
+                               num_splits, workspace, out, lse, stream)
+    _check_kv_new(kv_new, kcache, block_table)
+    if kv_new.shape[1] != q.shape[1]:
+        raise MlaError("kv_new and q must have the same s_q")
+    _check(lib.mla_decode_fwd_append(args[0], _ptr(kv_new), *args[1:]), "mla_decode_fwd_append")
     return out, lse
 
 

@@ -9,6 +9,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -36,6 +37,10 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Test hook (mla_test_withhold_q_ready): read by every launch that follows.
+std::atomic<int> g_withhold_q_ready{0};
+std::atomic<long long> g_wait_cycles{0};
 
 int ensure_encode() {
   if (g_encode) return MLA_OK;
@@ -202,20 +207,31 @@ int prepare(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int dtype
   p->num_parts = num_sm_parts;
   p->causal = causal;
   p->scale_log2 = softmax_scale * 1.4426950408889634f;
+  const long long wc = g_wait_cycles.load();
+  p->wait_cycles = wc > 0 ? wc : kDefaultWaitCycles;
+  p->withhold_q_ready = g_withhold_q_ready.load();
   p->block_table = nullptr;
   p->block_table_stride = 0;
   p->num_pages = 0;
   return MLA_OK;
 }
 
-int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
-                 int64_t block_table_stride, const DecodeParams& base, int dtype, cudaStream_t stream) {
+// Checks of the arguments only the split-KV kernel reads.
+int check_cache_args(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                     int64_t block_table_stride) {
   if (!q || !kcache || !block_table) return MLA_ERR_INVALID_ARG;
   if (num_pages < 1 || block_table_stride < 1) return MLA_ERR_INVALID_ARG;
   if (num_pages > (int64_t(1) << 31) - 1) return MLA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kcache)) return MLA_ERR_INVALID_ARG;
+  return MLA_OK;
+}
+
+int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                 int64_t block_table_stride, const DecodeParams& base, int dtype, cudaStream_t stream) {
+  int rc = check_cache_args(q, kcache, num_pages, block_table, block_table_stride);
+  if (rc != MLA_OK) return rc;
   int dev = 0;
-  int rc = current_device(&dev);
+  rc = current_device(&dev);
   if (rc != MLA_OK) return rc;
   if ((rc = ensure_device(dev)) != MLA_OK) return rc;
   if ((rc = ensure_encode()) != MLA_OK) return rc;
@@ -241,6 +257,18 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
 
 namespace mla {
 void set_last_cuda_error(int err) { g_last_cuda_error = err; }
+
+int check_decode_args(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                      int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                      int dtype, float softmax_scale, int causal, const int32_t* tile_sched_metadata,
+                      const int32_t* num_splits, int num_sm_parts, void* workspace, size_t workspace_bytes,
+                      void* out, float* lse) {
+  DecodeParams p;
+  int rc = prepare(cache_seqlens, batch, s_q, h_q, dtype, causal, tile_sched_metadata, num_splits, num_sm_parts,
+                   workspace, workspace_bytes, out, lse, softmax_scale, &p);
+  if (rc != MLA_OK) return rc;
+  return check_cache_args(q, kcache, num_pages, block_table, block_table_stride);
+}
 }  // namespace mla
 
 extern "C" {
@@ -258,7 +286,15 @@ const char* mla_status_string(int status) {
 
 int mla_last_cuda_error(void) { return g_last_cuda_error; }
 
-int mla_version(void) { return 100; }
+int mla_version(void) { return 200; }
+
+int mla_test_withhold_q_ready(int enable, long long wait_cycles) {
+  if (enable != 0 && enable != 1) return MLA_ERR_INVALID_ARG;
+  if (wait_cycles < 0) return MLA_ERR_INVALID_ARG;
+  g_withhold_q_ready.store(enable);
+  g_wait_cycles.store(wait_cycles);
+  return MLA_OK;
+}
 
 
 int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts) {
@@ -335,6 +371,44 @@ int mla_decode_fwd(const void* q, const void* kcache, int64_t num_pages, const i
   if ((rc = splitkv_impl(q, kcache, num_pages, block_table, block_table_stride, p, dtype, st)) != MLA_OK) return rc;
   cudaError_t e = launch_combine(dtype == MLA_BF16, p, st);
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
+}
+
+int mla_append_kv(const void* kv_new, void* kcache, int64_t num_pages, const int32_t* block_table,
+                  int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!kv_new || !kcache || !block_table || !cache_seqlens || !workspace) return MLA_ERR_INVALID_ARG;
+  if (batch < 1 || s_q < 1 || num_pages < 1 || block_table_stride < 1) return MLA_ERR_INVALID_ARG;
+  if (batch > kMaxBatch || s_q > kMaxRows) return MLA_ERR_UNSUPPORTED;
+  if (num_pages > (int64_t(1) << 31) - 1) return MLA_ERR_UNSUPPORTED;
+  if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(kv_new) || !aligned16(kcache) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MLA_ERR_INVALID_ARG;
+  if (workspace_bytes < kWsHeader) return MLA_ERR_WORKSPACE;
+  cudaError_t e = launch_append(kv_new, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch,
+                                s_q, static_cast<int*>(workspace), static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MLA_OK : cuda_fail(e);
+}
+
+int mla_decode_fwd_append(const void* q, const void* kv_new, void* kcache, int64_t num_pages,
+                          const int32_t* block_table, int64_t block_table_stride, const int32_t* cache_seqlens,
+                          int batch, int s_q, int h_q, int dtype, float softmax_scale, int causal,
+                          const int32_t* tile_sched_metadata, const int32_t* num_splits, int num_sm_parts,
+                          void* workspace, size_t workspace_bytes, void* out, float* lse, void* stream) {
+  int rc = check_decode_args(q, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch, s_q, h_q,
+                             dtype, softmax_scale, causal, tile_sched_metadata, num_splits, num_sm_parts, workspace,
+                             workspace_bytes, out, lse);
+  if (rc != MLA_OK) return rc;
+  if (!kv_new || !aligned16(kv_new)) return MLA_ERR_INVALID_ARG;
+  int dev = 0;
+  if ((rc = current_device(&dev)) != MLA_OK) return rc;
+  if ((rc = ensure_device(dev)) != MLA_OK) return rc;
+  if ((rc = ensure_encode()) != MLA_OK) return rc;
+  if ((rc = mla_append_kv(kv_new, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch, s_q,
+                          dtype, workspace, workspace_bytes, stream)) != MLA_OK)
+    return rc;
+  return mla_decode_fwd(q, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch, s_q, h_q,
+                        dtype, softmax_scale, causal, tile_sched_metadata, num_splits, num_sm_parts, workspace,
+                        workspace_bytes, out, lse, stream);
 }
 
 int mla_read_device_status(const void* workspace, void* stream, int32_t* flags) {

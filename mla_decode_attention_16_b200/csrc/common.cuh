@@ -20,9 +20,13 @@ constexpr int kTileRows = 128;            // query rows per MMA tile
 constexpr int kMaxRows = 1024;            // s_q * h_q supported (8 row tiles)
 constexpr int kMaxBatch = 16384;          // metadata kernel keeps lengths in smem
 
+// Default limit of every pipeline wait in the kernels: ~2 s at 1.9 GHz.
+constexpr long long kDefaultWaitCycles = 4000000000LL;
+
 // Device-side error bits (sticky, OR-ed into the first word of the workspace).
 constexpr int kDevErrTimeout = MLA_DEVERR_TIMEOUT;
 constexpr int kDevErrPage = MLA_DEVERR_PAGE_INDEX;
+constexpr int kDevErrAppendPos = MLA_DEVERR_APPEND_POS;
 
 // Workspace: [ error words | lse partials | o partials ], each 256-B aligned.
 constexpr size_t kWsHeader = 256;
@@ -51,6 +55,8 @@ struct DecodeParams {
   int batch, s_q, h_q, rows, m_tiles, num_parts;
   int causal;
   float scale_log2;  // softmax_scale * log2(e)
+  long long wait_cycles;  // limit of every pipeline wait, in SM clock cycles
+  int withhold_q_ready;   // test hook: 1 = the first chunk's "Q ready" arrival is never made
 };
 
 }  // namespace mla

@@ -23,6 +23,10 @@ const void* narrow_kernel_ptr(bool bf16, int np);
 cudaError_t launch_splitkv_narrow(bool bf16, const void* q, const CUtensorMap& kmap, const DecodeParams& p,
                                   cudaStream_t stream);
 cudaError_t launch_combine(bool bf16, const DecodeParams& p, cudaStream_t stream);
+// Copies kv_new [batch, s_q, 576] into cache positions L_b - s_q + s (programmatic dependent launch).
+cudaError_t launch_append(const void* kv_new, void* kcache, int64_t num_pages, const int32_t* block_table,
+                          int64_t bt_stride, const int32_t* seqlens, int batch, int s_q, int* err,
+                          cudaStream_t stream);
 int metadata_smem_bytes(int batch, int num_parts);
 constexpr int kMaxParts = 1024;  // partitions the metadata kernel stages in shared memory
 const void* metadata_kernel_ptr();
@@ -30,5 +34,12 @@ cudaError_t launch_metadata(const int32_t* seqlens, int batch, int num_parts, in
                             cudaStream_t stream);
 // Records a cudaError_t for mla_last_cuda_error() (per thread).
 void set_last_cuda_error(int err);
+// Every host-side check mla_decode_fwd makes, with nothing enqueued: MLA_OK or the status that
+// mla_decode_fwd would return for these arguments before launching anything.
+int check_decode_args(const void* q, const void* kcache, int64_t num_pages, const int32_t* block_table,
+                      int64_t block_table_stride, const int32_t* cache_seqlens, int batch, int s_q, int h_q,
+                      int dtype, float softmax_scale, int causal, const int32_t* tile_sched_metadata,
+                      const int32_t* num_splits, int num_sm_parts, void* workspace, size_t workspace_bytes,
+                      void* out, float* lse);
 
 }  // namespace mla

@@ -1,10 +1,11 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05
 // (TMEM alloc / MMA / ld / st / commit), cluster shared memory, PDL.
 //
-// Every wait here is bounded: a wait that does not complete within
-// kWaitCycles cycles records MLA_DEV_TIMEOUT in the caller's error word, raises
-// the CTA's abort flag and returns, so a broken pipeline ends instead of
-// hanging the GPU.  Once the abort flag is up, every later wait returns at once.
+// Every wait here is bounded: a wait that does not complete within the CTA's
+// wait limit (WaitCtl::limit clock cycles, ~2 s by default) records
+// MLA_DEVERR_TIMEOUT in the caller's error word, raises the CTA's abort flag
+// and returns, so a broken pipeline ends instead of hanging the GPU.  Once the
+// abort flag is up, every later wait returns at once.
 #pragma once
 
 #include <cstdint>
@@ -14,7 +15,17 @@
 namespace mla {
 namespace ptx {
 
-constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+// Abort state of a CTA, kept in its shared memory: the flag every bounded wait raises and tests,
+// and the wait limit in clock cycles.
+struct WaitCtl {
+  int abort;
+  int pad;
+  long long limit;
+};
+__device__ __forceinline__ bool aborted(const WaitCtl* c) {
+  return *reinterpret_cast<const volatile int*>(&c->abort) != 0;
+}
+__device__ __forceinline__ void raise_abort(WaitCtl* c) { *reinterpret_cast<volatile int*>(&c->abort) = 1; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -80,17 +91,18 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // The abort flag and the clock are looked at only every 16 polls, so a waiting
 // warp issues little besides the polls themselves.
 template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err_word, int err_code) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, WaitCtl* ctl, int* err_word,
+                                          int err_code) {
   if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-  if (*abort_flag) return false;
+  if (aborted(ctl)) return false;
   const long long t0 = clock64();
+  const long long limit = ctl->limit;
   for (uint32_t n = 1;; ++n) {
     if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((n & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *abort_flag = 1;
+      if (aborted(ctl)) return false;
+      if (clock64() - t0 > limit) {
+        raise_abort(ctl);
         if (err_word) atomicOr(err_word, err_code);
         return false;
       }
@@ -100,10 +112,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // Bounded wait that ignores the abort flag (used to drain in-flight async work
 // before teardown).
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, long long limit) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

@@ -109,7 +109,7 @@ enum Bar {
   kNumBars
 };
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemUsed = kOffMisc + 16;
+constexpr int kSmemUsed = kOffMisc + 8 + sizeof(WaitCtl);
 constexpr int kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  WaitCtl* wctl = reinterpret_cast<WaitCtl*>(smem + kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool two = i >= kXchg && i < kXchg + 8;
       mbar_init(bar(i), eight ? static_cast<uint32_t>(kSmWarps) : two ? 2u : 1u);
     }
-    *abort_flag = 0;
+    wctl->abort = 0;
+    wctl->limit = p.wait_cycles;
     for (int i = 0; i < kSmWarps; ++i) mbar_arrive_expect_tx(bar(kXFull + i), kXWarp);  // arm phase 0
     fence_mbar_init();
   }
@@ -241,13 +242,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         return x.valid ? p.block_table[static_cast<int64_t>(x.req) * p.block_table_stride + x.blk] : 0;
       };
       int page_next = page_of(w);
-      for (uint32_t it = 0; w.valid && !*abort_flag; ++it) {
+      uint32_t it = 0;
+      int q_chunks = 0;  // Q column boxes requested so far (one per chunk)
+      for (; w.valid && !aborted(wctl); ++it) {
         const int st = it % kStages;
         int page = page_next;
         Walk nx = w;
         nx.next(p);
         page_next = page_of(nx);  // the next block's page index is read while this stage frees up
-        mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        if (!mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, wctl, err, kDevErrTimeout)) break;
         if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
           atomicOr(err, kDevErrPage);
           atomicCAS(err + 1, 0, page == 0 ? -1 : page);
@@ -260,12 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d_hint(dst + 4 * kKBox, &krmap, bar(kKvFull + st), 512 + 32 * crank, 0, page, evict_first);
         if (w.first()) {
           // the chunk's Q columns 512 + 32c .., once the previous chunk's last Q.K^T has read the old ones
-          mbar_wait(bar(kQEmpty), (w.chunk & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-          mbar_arrive_expect_tx(bar(kQrFull), kQrBox);
-          tma_load_2d(sbase + kOffQR, &qrmap, bar(kQrFull), 512 + 32 * crank, w.req * R + mtile * kTileRows);
+          if (mbar_wait(bar(kQEmpty), (w.chunk & 1) ^ 1, wctl, err, kDevErrTimeout)) {
+            mbar_arrive_expect_tx(bar(kQrFull), kQrBox);
+            tma_load_2d(sbase + kOffQR, &qrmap, bar(kQrFull), 512 + 32 * crank, w.req * R + mtile * kTileRows);
+            ++q_chunks;
+          }
         }
         w = nx;
       }
+      // Before the CTA can exit, every TMA load issued above must have landed: wait (bounded, abort
+      // or not) for the last phase of each stage and of the Q box.  A phase the MMA warp already
+      // consumed has completed, so the wait returns at once; only an abort leaves one pending.
+      for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+        mbar_wait_drain(bar(kKvFull + j % kStages), (j / kStages) & 1, wctl->limit);
+      if (q_chunks > 0) mbar_wait_drain(bar(kQrFull), (q_chunks - 1) & 1, wctl->limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -341,10 +352,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_qk();
         } else {
           if ((++polls & 15u) == 0) {
-            if (*abort_flag) break;
+            if (aborted(wctl)) break;
             const long long now = clock64();
-            if (now - idle_since > kWaitCycles) {
-              *abort_flag = 1;
+            if (now - idle_since > wctl->limit) {
+              raise_abort(wctl);
               atomicOr(err, kDevErrTimeout);
               break;
             }
@@ -354,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         idle_since = clock64();
       }
       umma_commit(bar(kDrain));
-      mbar_wait_drain(bar(kDrain), 0);
+      mbar_wait_drain(bar(kDrain), 0, wctl->limit);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ Q to TMEM, exchange, softmax, correction, epilogue
@@ -390,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t xb = bar(kXchg + 2 * q4 + par);
       const int idx = par * 4 * kTileRows + (2 * static_cast<int>(crank) + sub) * kTileRows + row;
       slots[idx] = v;
-      st_async_b32(mapa(sbase + kOffRed + 4 * idx, peer), mapa(xb, peer), v);
+      if (!aborted(wctl)) st_async_b32(mapa(sbase + kOffRed + 4 * idx, peer), mapa(xb, peer), v);
       __syncwarp();
       if (lane == 0) {
         if (sub == 0)
@@ -401,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto xchg_wait = [&](float (&v)[4]) {
       const int par = xc & 1;
-      mbar_wait(bar(kXchg + 2 * q4 + par), (xc >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      mbar_wait(bar(kXchg + 2 * q4 + par), (xc >> 1) & 1, wctl, err, kDevErrTimeout);
       const float* slot = slots + par * 4 * kTileRows + row;
 #pragma unroll
       for (int k = 0; k < 4; ++k) v[k] = slot[k * kTileRows];
@@ -446,12 +457,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       nx.next(p);
       const bool new_q = nx.valid && nx.chunk != wu.chunk;
       if (new_q && active) prefetch_q(nx.req);  // into L1 while the scores finish
-      mbar_wait(bar(kSFull + b), (u >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      mbar_wait(bar(kSFull + b), (u >> 1) & 1, wctl, err, kDevErrTimeout);
       __syncwarp();  // reconverge before the warp-collective tcgen05 ops
+      if (aborted(wctl)) return;  // the same for every lane after the warp barrier: nothing is sent
       tc_fence_after();
       if (new_q) {
         // the Q.K^T of block u was the chunk's last: the Q columns are free
-        mbar_wait(bar(kQEmpty), wu.chunk & 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kQEmpty), wu.chunk & 1, wctl, err, kDevErrTimeout);
         __syncwarp();
         tc_fence_after();
         if (active) store_q(nx.req);
@@ -469,13 +481,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < 4; ++g)
           pack24(r[4 * g], r[4 * g + 1], r[4 * g + 2], r[4 * g + 3], w[3 * g], w[3 * g + 1], w[3 * g + 2]);
         // the peer's receive slot of this warp is free once the peer has combined block u - 1
-        if (lane == 0) mbar_wait<true>(bar(kXEmpty + sm), (u & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        if (lane == 0) mbar_wait<true>(bar(kXEmpty + sm), (u & 1) ^ 1, wctl, err, kDevErrTimeout);
         __syncwarp();
         const uint32_t dst = mapa(sbase + kOffRcv + sm * kXWarp + lane * kRowBytes, peer);
         const uint32_t rb = mapa(bar(kXFull + sm), peer);
+        if (!aborted(wctl))
 #pragma unroll
-        for (int j = 0; j < 3; ++j)
-          st_async_v4(dst + 16 * j, rb, __uint_as_float(w[4 * j]), __uint_as_float(w[4 * j + 1]),
+          for (int j = 0; j < 3; ++j)
+            st_async_v4(dst + 16 * j, rb, __uint_as_float(w[4 * j]), __uint_as_float(w[4 * j + 1]),
                       __uint_as_float(w[4 * j + 2]), __uint_as_float(w[4 * j + 3]));
       }
     };
@@ -487,21 +500,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (active) store_q(wu.req);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kQtFull));
+      if (lane == 0 && !(p.withhold_q_ready && sm == 0)) mbar_arrive(bar(kQtFull));
       send_partial(0, wu);
       wu.next(p);
     }
     uint32_t u = 1;
     float m = -INFINITY, l = 0.f;  // m: exponent reference (log2 units), l: this thread's keys' row sum relative to it
     for (uint32_t t = 0; wt.valid; ++t, wt.next(p)) {
-      if (*abort_flag) break;
+      if (aborted(wctl)) break;
       // ---- block t: own partial + the peer's, then release the score buffer.  Only this CTA
       // computes the scores of its keys (the peer gets their P), so its own partial keeps full
       // precision; the peer's arrives rounded to 24 bits.
       const int b = t & 1;
       float x[kOwnN];
       if (active) {
-        mbar_wait<true>(bar(kXFull + sm), t & 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait<true>(bar(kXFull + sm), t & 1, wctl, err, kDevErrTimeout);
         __syncwarp();
         uint32_t r[16];
         tmem_ld16(t_lane + kColS + 64 * b + own_col, r);
@@ -558,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // reads are complete: arm the slot's next phase, then let the peer refill it (a relaxed
           // arrive; a release at cluster scope costs ~1000 cycles here)
           mbar_arrive_expect_tx(bar(kXFull + sm), kXWarp);
-          mbar_arrive_cluster_relaxed_after(mapa(bar(kXEmpty + sm), peer), mx);
+          if (!aborted(wctl)) mbar_arrive_cluster_relaxed_after(mapa(bar(kXEmpty + sm), peer), mx);
         }
         xchg_post(mx);
       }
@@ -568,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++u;
       }
       if (!active) {
-        mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kPEmpty), (t & 1) ^ 1, wctl, err, kDevErrTimeout);
         __syncwarp();
         if (lane == 0) {
           if (sm == 0)
@@ -607,9 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // P (this thread's 16 keys of the row), once this CTA's previous P.V has read P (so O also
         // holds every earlier block); then tell the peer it may copy its part of P here
-        mbar_wait(bar(kPEmpty), (t & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kPEmpty), (t & 1) ^ 1, wctl, err, kDevErrTimeout);
         if (lane == 0) {
-          mbar_arrive_cluster_relaxed_after(mapa(bar(kPeerFree + sm), peer), 0.f);
+          if (!aborted(wctl)) mbar_arrive_cluster_relaxed_after(mapa(bar(kPeerFree + sm), peer), 0.f);
           bulk_wait_read_all();  // this piece's copy of the previous block is done
         }
         __syncwarp();
@@ -624,9 +637,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) {
           // the peer's P.V of the previous block has read its P too
-          mbar_wait<true>(bar(kPeerFree + sm), t & 1, abort_flag, err, kDevErrTimeout);
-          bulk_copy_to_peer(mapa(p_piece, peer), p_piece, 1024, mapa(bar(kPFull), peer));
-          bulk_commit_group();
+          mbar_wait<true>(bar(kPeerFree + sm), t & 1, wctl, err, kDevErrTimeout);
+          if (!aborted(wctl)) {
+            bulk_copy_to_peer(mapa(p_piece, peer), p_piece, 1024, mapa(bar(kPFull), peer));
+            bulk_commit_group();
+          }
         }
         if (__any_sync(0xffffffffu, resc)) {
           // only blocks after the chunk's first can move an established reference, so O holds
@@ -663,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         xchg_wait(v);
         lt = (v[0] + v[1]) + (v[2] + v[3]);  // the same order in both CTAs
       }
-      mbar_wait(bar(kOFinal), wt.chunk & 1, abort_flag, err, kDevErrTimeout);
+      mbar_wait(bar(kOFinal), wt.chunk & 1, wctl, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
       if (active) {

@@ -81,7 +81,7 @@ struct Layout {
   static constexpr int kRedFloats = 2 * NP + 2 + 2 * NP + 2 * NP;
   static constexpr int kOffBar = (kOffRed + kRedFloats * 4 + 7) / 8 * 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr int kSmemBytes = kOffMisc + 8 + sizeof(WaitCtl) + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 0;     // O: 2 halves of 256 values x 64 columns (see umma_ws_ss)
@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kOffBar + 8 * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
+  WaitCtl* wctl = reinterpret_cast<WaitCtl*>(smem + Lay::kOffMisc + 8);
   float* s_alpha = reinterpret_cast<float*>(smem + Lay::kOffRed);          // [2][NP]
   volatile int* s_flag = reinterpret_cast<volatile int*>(s_alpha + 2 * NP);  // [2]
   float* s_lsum = s_alpha + 2 * NP + 2;                                   // [2][NP]
@@ -148,7 +148,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool four = i == kPFull || i == kPFull + 1 || i == kOEmpty || i == kOEmpty + 1;
       mbar_init(bar(i), four ? 4u : 1u);
     }
-    *abort_flag = 0;
+    wctl->abort = 0;
+    wctl->limit = p.wait_cycles;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -177,15 +178,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       int cur = br;
       Chunk ch;
-      while (!*abort_flag && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
+      while (!aborted(wctl) && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
         const int32_t* bt = p.block_table + static_cast<int64_t>(ch.req) * p.block_table_stride;
         int page_next = bt[ch.lo];
         for (int blk = ch.lo; blk < ch.hi; ++blk, ++it) {
-          if (*abort_flag) break;
+          if (aborted(wctl)) break;
           const int st = it % kStages;
           int page = page_next;
           if (blk + 1 < ch.hi) page_next = bt[blk + 1];  // read while this stage frees up
-          mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          if (!mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, wctl, err, kDevErrTimeout)) break;
           if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
             atomicOr(err, kDevErrPage);
             atomicCAS(err + 1, 0, page == 0 ? -1 : page);
@@ -197,6 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                              0, page, evict_first);
         }
       }
+      // Before the CTA can exit, every page load issued above must have landed: wait (bounded, abort
+      // or not) for the last phase of each stage.  A phase the MMA warp already consumed has
+      // completed, so the wait returns at once; only an abort leaves one pending.
+      for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+        mbar_wait_drain(bar(kKvFull + j % kStages), (j / kStages) & 1, wctl->limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -208,8 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = itp % kStages;
         const int b = itp & 1;
         const int ob = chunk % kOBufs;
-        if (jjp == 0) mbar_wait(bar(kOEmpty + ob), ((chunk / kOBufs) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
-        mbar_wait(bar(kPFull + b), (itp >> 1) & 1, abort_flag, err, kDevErrTimeout);
+        if (jjp == 0) mbar_wait(bar(kOEmpty + ob), ((chunk / kOBufs) & 1) ^ 1, wctl, err, kDevErrTimeout);
+        mbar_wait(bar(kPFull + b), (itp >> 1) & 1, wctl, err, kDevErrTimeout);
         tc_fence_after();
         const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
         const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
@@ -232,16 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       int cur = br;
       Chunk ch;
-      while (!*abort_flag && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
+      while (!aborted(wctl) && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
         const int nb = ch.hi - ch.lo;
         const int qpar = chunk & 1;
-        mbar_wait(bar(kQFull + qpar), (chunk >> 1) & 1, abort_flag, err, kDevErrTimeout);
+        mbar_wait(bar(kQFull + qpar), (chunk >> 1) & 1, wctl, err, kDevErrTimeout);
         tc_fence_after();
         for (int jj = 0; jj < nb; ++jj) {
           const uint32_t itc = it + jj;
           const int st = itc % kStages;
-          mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, abort_flag, err, kDevErrTimeout);
-          mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, wctl, err, kDevErrTimeout);
+          mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, wctl, err, kDevErrTimeout);
           tc_fence_after();
           const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
 #pragma unroll 1
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++chunk;
       }
       umma_commit(bar(kDrain));
-      mbar_wait_drain(bar(kDrain), 0);
+      mbar_wait_drain(bar(kDrain), 0, wctl->limit);
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ softmax (one warp per chunk) + O rescale
@@ -286,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t itc = it + jj;
         const int b = itc & 1;
         if (smx) {
-          mbar_wait(bar(kSFull), itc & 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kSFull), itc & 1, wctl, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
           float x[64];
@@ -336,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool any_resc = __any_sync(0xffffffffu, resc);
           if (r < NP) s_alpha[b * NP + r] = alpha;
           if (lane == 0) s_flag[b] = any_resc ? 1 : 0;
-          mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
           if (r < NP) {
             // P row r: 64 keys = 128 bytes, 16-byte chunks XOR-swizzled by row (128-byte swizzle)
             uint8_t* prow = smem + Lay::kOffP + b * Lay::kPBytes + r * 128;
@@ -349,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_bar_sync(1, 128);
         if (s_flag[b] && jj > 0) {
-          mbar_wait(bar(kODone), (itc - 1) & 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kODone), (itc - 1) & 1, wctl, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
           // lane r of every quadrant holds row r: 64 columns of each half of its values
@@ -374,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // this stats slot was last used by chunk - 2; with two O buffers its epilogue may still
         // be reading it (with one buffer the MMA order already guarantees it finished)
         if (kOBufs == 2 && chunk >= 2)
-          mbar_wait(bar(kOEmpty + par), ((chunk >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+          mbar_wait(bar(kOEmpty + par), ((chunk >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
         if (r < NP) {
           s_lsum[par * NP + r] = l;
           s_mref[par * NP + r] = m;
@@ -392,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = lane;
     auto load_q = [&](const Chunk& c, uint32_t idx) {
       // Q rows of chunk idx into lane quadrant idx & 1 (this warp's quadrant)
-      mbar_wait(bar(kQEmpty + (idx & 1)), ((idx >> 1) & 1) ^ 1, abort_flag, err, kDevErrTimeout);
+      mbar_wait(bar(kQEmpty + (idx & 1)), ((idx >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
       const uint4* qrow = reinterpret_cast<const uint4*>(
@@ -414,13 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(kQFull + (idx & 1)));
+      if (lane == 0 && !(p.withhold_q_ready && idx == 0)) mbar_arrive(bar(kQFull + (idx & 1)));
     };
     auto epilogue = [&](const Chunk& c, uint32_t idx) {
       const int ob = idx % kOBufs;
       const int par = idx & 1;
-      mbar_wait(bar(kOFinal + ob), (idx / kOBufs) & 1, abort_flag, err, kDevErrTimeout);
-      mbar_wait(bar(kStats + par), (idx >> 1) & 1, abort_flag, err, kDevErrTimeout);
+      mbar_wait(bar(kOFinal + ob), (idx / kOBufs) & 1, wctl, err, kDevErrTimeout);
+      mbar_wait(bar(kStats + par), (idx >> 1) & 1, wctl, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
       const bool whole = (c.lo == 0 && c.hi == c.n);

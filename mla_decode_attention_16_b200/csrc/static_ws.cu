@@ -74,6 +74,12 @@ extern "C" int mla_decode_fwd_static_ws(const void* q, const void* kcache, int64
   if (need > kStaticScratchBytes) return MLA_ERR_WORKSPACE;  // larger than the built-in scratch
   void* scratch = nullptr;
   if ((rc = scratch_on_current_device(&scratch)) != MLA_OK) return rc;
+  // Every check the forward makes runs before the header is cleared, so a rejected call enqueues
+  // nothing (and leaves the error word of an earlier call untouched).
+  rc = mla::check_decode_args(q, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch, s_q,
+                              h_q, dtype, softmax_scale, causal, tile_sched_metadata, num_splits, num_sm_parts,
+                              scratch, kStaticScratchBytes, out, lse);
+  if (rc != MLA_OK) return rc;
   // The scratch keeps whatever the previous call left.  Only the error header
   // must start at zero; every partial is written before it is read.
   cudaError_t e = cudaMemsetAsync(scratch, 0, mla::kWsHeader, static_cast<cudaStream_t>(stream));
@@ -84,4 +90,12 @@ extern "C" int mla_decode_fwd_static_ws(const void* q, const void* kcache, int64
   return mla_decode_fwd(q, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch, s_q, h_q,
                         dtype, softmax_scale, causal, tile_sched_metadata, num_splits, num_sm_parts, scratch,
                         kStaticScratchBytes, out, lse, stream);
+}
+
+extern "C" int mla_static_ws_read_device_status(void* stream, int32_t* flags) {
+  if (!flags) return MLA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  int rc = scratch_on_current_device(&scratch);
+  if (rc != MLA_OK) return rc;
+  return mla_read_device_status(scratch, stream, flags);
 }

@@ -16,6 +16,9 @@ mla_ref.mla_partial_ref / mla_ref.merge_partials_ref
 sched_ref.tile_schedule_ref
     the tile scheduler (per-partition quota + greedy in-order walk), pure Python
     integers.
+append_ref.append_kv_ref / append_ref.decode_with_append_ref
+    the new tokens' rows written into their page slots (the step before a
+    decode), and "append, then decode".
 
 Sources (pages, by title and section)
 -------------------------------------
@@ -33,6 +36,7 @@ Sources (pages, by title and section)
   ``return_softmax_lse`` conventions of a KV-cache attention call.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(``tests/append_pins.py`` for the append)
 (closed forms, invariants, brute force, an independent library special case)
 and ``tests/test_oracle_mutants.py`` (planted mistakes must fail a pin).
 """
@@ -47,3 +51,4 @@ from .mla_ref import (  # noqa: F401
     visible_key_count,
 )
 from .sched_ref import FIXED_OVERHEAD_BLOCKS, tile_schedule_ref  # noqa: F401
+from .append_ref import append_kv_ref, decode_with_append_ref  # noqa: F401

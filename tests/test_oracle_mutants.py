@@ -12,8 +12,10 @@ import types
 
 import pytest
 
+import oracle.append_ref as app
 import oracle.mla_ref as ref
 import oracle.sched_ref as sched
+from append_pins import ALL_APPEND_PINS
 from oracle_pins import ALL_PINS
 from sched_pins import ALL_SCHED_PINS
 
@@ -57,6 +59,18 @@ SCHED_MUTANTS = {
                                        "            nxt = first_of_part[p]\n        begins[p] = nxt if p in first_of_part else (b, 0, 0)"),
 }
 
+APPEND_MUTANTS = {
+    "position off by one": ("j = L - s_q + s  #", "j = L - s_q + s + 1  #"),
+    "lengths exclude the new tokens": ("j = L - s_q + s  #", "j = L + s  #"),
+    "new tokens in reverse order": ("out[page, slot, 0, :] = kv_new[r, s, :]",
+                                    "out[page, slot, 0, :] = kv_new[r, s_q - 1 - s, :]"),
+    "page by modulo": ("page = int(block_table[r, j // PAGE])", "page = int(block_table[r, j % PAGE])"),
+    "slot by division": ("slot = j % PAGE", "slot = j // PAGE"),
+    "first request's table": ("page = int(block_table[r, j // PAGE])", "page = int(block_table[0, j // PAGE])"),
+    "writes into the input": ("out = kcache.clone()", "out = kcache"),
+    "short request wraps around": ("            if j < 0:\n                continue\n", ""),
+}
+
 
 def _mutant(module: types.ModuleType, edits) -> types.ModuleType:
     """Copy of ``module`` with each (old, new) text substitution applied."""
@@ -92,6 +106,12 @@ def _caught(pins, mod) -> list:
 def test_attention_mutant_is_caught(name):
     mod = _mutant(ref, ATTN_MUTANTS[name])
     assert _caught(ALL_PINS, mod), f"mutant '{name}' passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(APPEND_MUTANTS))
+def test_append_mutant_is_caught(name):
+    mod = _mutant(app, APPEND_MUTANTS[name])
+    assert _caught(ALL_APPEND_PINS, mod), f"mutant '{name}' passed every pin"
 
 
 @pytest.mark.parametrize("name", sorted(SCHED_MUTANTS))

@@ -9,3 +9,12 @@ from oracle_pins import ALL_PINS
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
 def test_oracle_pin(pin):
     pin(ref)
+
+
+import oracle.append_ref as app  # noqa: E402
+from append_pins import ALL_APPEND_PINS  # noqa: E402
+
+
+@pytest.mark.parametrize("pin", ALL_APPEND_PINS, ids=lambda p: p.__name__)
+def test_append_oracle_pin(pin):
+    pin(app)
