@@ -153,11 +153,24 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
-def kernel_of(rows: int):
+KERNELS = {  # variant -> (kernel name, source file)
+    "few-rows-one-cta": ("splitkv_narrow_kernel", "splitkv_narrow.cu"),
+    "few-rows-pair": ("splitkv_npair_kernel", "splitkv_npair.cu"),
+    "row-tile-pair": ("splitkv_pair_kernel", "splitkv.cu"),
+}
+
+
+def variant_of(rows: int, variant: str = "auto") -> str:
+    """The split-KV kernel variant the library runs for s_q * h_q = rows (its default choice for
+    "auto": the one-CTA few-row kernel up to 32 rows, the row-tile pair kernel above)."""
+    if variant != "auto":
+        return variant
+    return "few-rows-one-cta" if rows <= 32 else "row-tile-pair"
+
+
+def kernel_of(rows: int, variant: str = "auto"):
     """(name, source file) of the split-KV kernel the library runs for s_q * h_q = rows."""
-    if rows <= 32:
-        return "splitkv_narrow_kernel", "splitkv_narrow.cu"
-    return "splitkv_pair_kernel", "splitkv.cu"
+    return KERNELS[variant_of(rows, variant)]
 
 
 def profile_traffic(name: str, kernel: str, source: str):
@@ -266,12 +279,14 @@ def init_dist():
     return world, rank, torch.device("cuda", torch.cuda.current_device())
 
 
-def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, cpu_seconds: float):
+def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, cpu_seconds: float,
+                variant: str = "auto"):
     """Device throughput, split-KV kernel time, end-to-end throughput (and, on rank 0 of a 1-GPU run
     with cpu_seconds > 0, the CPU oracle's) of one workload.  Every rank makes the same collective
     calls in the same order; rank 0 gets the result dict, the others None."""
     import mla_decode_attention_16_b200 as mla
 
+    mla.mla_set_kernel_variant(variant)
     unit = unit_of(name)
     w = WORKLOADS[name]
     if rank == 0:
@@ -423,10 +438,11 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
         achieved = cost["flops"] / kern_s / 1e12
         peak = float(peaks["bf16_tflops"])  # fp16 dense tensor rate equals bf16 on this part
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
-    kname, ksrc = kernel_of(rows)
+    kname, ksrc = kernel_of(rows, variant)
     roof["traffic"] = profile_traffic(name, kname, ksrc)
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["kernel"] = kname
+    roof["variant"] = variant_of(rows, variant)
     roof["kernel_us"] = kern_s * 1e6
     roof["algorithmic_per_launch"] = cost["bytes"] if unit == "GB/s" else cost["flops"]
     res = {
@@ -446,6 +462,92 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
     return res
 
 
+# ----------------------------------------------------------------------------- row-count study
+SWEEP_H = (16, 32, 64, 128)
+SWEEP_S = (1, 2, 4, 8)
+
+
+def sweep_shapes():
+    """(h_q, s_q) pairs of the row-count study: every combination, s_q * h_q up to 1024 rows."""
+    return [(h, sq) for h in SWEEP_H for sq in SWEEP_S if h * sq <= 1024]
+
+
+def variants_for(rows: int):
+    """Kernel variants that can run s_q * h_q = rows query rows."""
+    if rows <= 32:
+        return ["few-rows-one-cta", "few-rows-pair", "row-tile-pair"]
+    return ["row-tile-pair"]
+
+
+def binding_roof(cost: dict, peaks: dict):
+    """(seconds at the binding roofline, which roof) for one call: the larger of HBM time and
+    tensor time at the measured peaks."""
+    t_hbm = cost["bytes"] / (float(peaks["hbm_gbs"]) * 1e9)
+    t_tc = cost["flops"] / (float(peaks["bf16_tflops"]) * 1e12)
+    return (t_hbm, "hbm") if t_hbm >= t_tc else (t_tc, "tensor")
+
+
+def run_sweep(args):
+    """Split-KV kernel time of every kernel variant over h_q x s_q (batch 64, 4096 cached tokens per
+    request, bf16, causal when s_q > 1): one JSON line per (shape, variant) with the fraction of the
+    binding roofline, then one line naming the fastest variant per row count."""
+    import mla_decode_attention_16_b200 as mla
+    from workloads import make_case
+
+    world, rank, dev = init_dist()
+    peaks, _ = load_peaks()
+    best = {}
+    for h, sq in sweep_shapes():
+        rows = h * sq
+        inp = make_case(64, sq, h, [4096] * 64, causal=sq > 1, seed=5000 + rows + h)
+        lens = [4096] * 64
+        cost = algorithmic_cost(lens, sq, h)
+        q = inp.q.to(dev)
+        caches = [inp.kcache.to(dev), inp.kcache.to(dev)]
+        bt, sl = inp.block_table.to(dev), inp.cache_seqlens.to(dev)
+        out = torch.empty(64, sq, h, 512, dtype=q.dtype, device=dev)
+        lse = torch.empty(64, h, sq, dtype=torch.float32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+        for variant in variants_for(rows):
+            mla.mla_set_kernel_variant(variant)
+            parts = mla.mla_get_num_sm_parts(rows, dev.index)
+            meta, ns = mla.mla_get_metadata(sl, rows, parts)
+            ws = mla.alloc_workspace(64, rows, parts, dev)
+            for i in range(max(3, args.warmup)):
+                mla.mla_splitkv_fwd(q, caches[i & 1], bt, sl, inp.softmax_scale, inp.causal, meta, ns, ws, out, lse,
+                                    stream=stream)
+            torch.cuda.synchronize(dev)
+            n = max(3, min(args.steps, 50))
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            for i, (a, z) in enumerate(evs):
+                a.record(stream)
+                mla.mla_splitkv_fwd(q, caches[i & 1], bt, sl, inp.softmax_scale, inp.causal, meta, ns, ws, out, lse,
+                                    stream=stream)
+                z.record(stream)
+            torch.cuda.synchronize(dev)
+            flags = mla.mla_read_device_status(ws, stream)
+            if flags[0] != 0:
+                raise RuntimeError(f"sweep h_q {h} s_q {sq} {variant}: device error flags {flags}")
+            secs = statistics.median(a.elapsed_time(z) for a, z in evs) / 1000.0
+            roof_s, bound = binding_roof(cost, peaks)
+            line = {"mode": "sweep", "h_q": h, "s_q": sq, "rows": rows, "variant": variant,
+                    "kernel": KERNELS[variant][0], "kernel_us": secs * 1e6, "gbps": cost["bytes"] / secs / 1e9,
+                    "tflops": cost["flops"] / secs / 1e12, "bound": bound, "frac": roof_s / secs,
+                    "config": "batch 64, 4096 cached tokens per request, bf16, causal when s_q > 1"}
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+            if rows not in best or secs < best[rows][1]:
+                best[rows] = (variant, secs)
+            del ws
+        del caches, q
+        torch.cuda.empty_cache()
+    mla.mla_set_kernel_variant("auto")
+    if rank == 0:
+        print(json.dumps({"mode": "sweep-best", "fastest": {str(r): v for r, (v, _) in sorted(best.items())}}),
+              flush=True)
+    return 0
+
+
 # workloads whose numbers join the headline line of a default run (the pages' h_q * s_q >= 128 configs)
 COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16"]
 
@@ -453,12 +555,12 @@ COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16"]
 def run_gpu(args, name: str, companions=()):
     world, rank, dev = init_dist()
     cpu_s = 0.0 if args.no_cpu_baseline else args.cpu_seconds
-    head = measure_gpu(name, args.steps, args.warmup, world, rank, dev, cpu_s)
+    head = measure_gpu(name, args.steps, args.warmup, world, rank, dev, cpu_s, args.variant)
     extra = {}
     for other in companions:
         torch.cuda.empty_cache()
         extra[other] = measure_gpu(other, min(args.steps, args.companion_steps), args.warmup, world, rank, dev,
-                                   0.0 if args.no_cpu_baseline else args.companion_cpu_seconds)
+                                   0.0 if args.no_cpu_baseline else args.companion_cpu_seconds, args.variant)
     if rank == 0:
         line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
@@ -482,12 +584,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + ["all"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS) + ["all", "sweep"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--companion-steps", type=int, default=200,
                     help="timed steps of each h_q*s_q >= 128 workload added to a default run's line")
     ap.add_argument("--companion-cpu-seconds", type=float, default=5.0)
+    ap.add_argument("--variant", default="auto",
+                    choices=["auto", "few-rows-one-cta", "few-rows-pair", "row-tile-pair"],
+                    help="split-KV kernel variant (default: the library's choice by row count)")
     ap.add_argument("--headline-only", action="store_true",
                     help="a default run measures only the headline workload")
     args = ap.parse_args(argv)
@@ -500,6 +605,8 @@ def main(argv=None):
             if rc:
                 return rc
         return 0
+    if args.workload == "sweep":
+        return run_sweep(args)
     if args.workload == "all":
         for name in [n for n in WORKLOADS if n != "tiny"]:
             rc = run_gpu(args, name)

@@ -79,10 +79,45 @@ int mla_last_cuda_error(void);
 int mla_version(void);
 
 /*
+ * Split-KV kernel variants.  Every variant computes the same result (within
+ * rounding); they differ in how the work maps onto the SMs.
+ *   MLA_KERNEL_AUTO              the default: the one-CTA few-row kernel for
+ *                                s_q * h_q <= 32, the row-tile kernel above
+ *   MLA_KERNEL_FEW_ROWS_ONE_CTA  rows <= 32: one CTA per partition loads whole
+ *                                pages (three 72 KB stages)
+ *   MLA_KERNEL_FEW_ROWS_PAIR     rows <= 32: a cluster of two CTAs per
+ *                                partition, each loading and contracting half
+ *                                of every page's columns and exchanging the
+ *                                partial scores (five 36 KB stages per CTA)
+ *   MLA_KERNEL_ROW_TILE_PAIR     any rows: a cluster of two CTAs per
+ *                                partition and 128-row tile, each owning half
+ *                                of the output columns
+ */
+#define MLA_KERNEL_AUTO 0
+#define MLA_KERNEL_FEW_ROWS_ONE_CTA 1
+#define MLA_KERNEL_FEW_ROWS_PAIR 2
+#define MLA_KERNEL_ROW_TILE_PAIR 3
+
+/*
+ * Process-wide choice of the split-KV kernel variant for the calls that follow
+ * (for tuning studies; the default, MLA_KERNEL_AUTO, needs no call).  The
+ * partition count depends on the variant, so call mla_get_num_sm_parts and
+ * mla_get_metadata again after changing it.  A forward call whose rows exceed
+ * what the chosen variant handles returns MLA_ERR_UNSUPPORTED.
+ * Returns MLA_ERR_INVALID_ARG for an unknown variant.  Host only.
+ */
+int mla_set_kernel_variant(int variant);
+
+/* The variant (MLA_KERNEL_FEW_ROWS_ONE_CTA .. MLA_KERNEL_ROW_TILE_PAIR) a call
+ * with `rows` = s_q * h_q would run now, or -1 if none can.  Host only. */
+int mla_get_kernel_variant(int rows);
+
+/*
  * Number of scheduler partitions for `rows` = s_q * h_q query rows per request
- * on `device`: one per SM when rows <= 32 (one CTA per partition), else the
- * number of co-resident CTA pairs divided by the number of 128-row tiles (one
- * CTA pair per partition and tile).  Host only; it queries the device's SM
+ * on `device` under the current kernel variant: one per SM for the one-CTA
+ * few-row kernel, one per co-resident CTA pair for the few-row pair kernel,
+ * and the co-resident CTA pairs divided by the number of 128-row tiles for the
+ * row-tile kernel.  Host only; it queries the device's SM
  * count and cluster occupancy once and caches it.  rows must be in [1, 1024].
  */
 int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts);

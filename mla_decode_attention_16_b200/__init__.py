@@ -38,6 +38,9 @@ __all__ = [
     "mla_append_kv",
     "mla_decode_fwd_append",
     "mla_read_device_status",
+    "mla_set_kernel_variant",
+    "mla_get_kernel_variant",
+    "KERNEL_VARIANTS",
     "HEAD_DIM_K",
     "HEAD_DIM_V",
     "PAGE_SIZE",
@@ -49,6 +52,8 @@ HEAD_DIM_V = 512
 PAGE_SIZE = 64
 META_INTS = 8
 _DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+# split-KV kernel variants (include/mla_decode.h, MLA_KERNEL_*)
+KERNEL_VARIANTS = {"auto": 0, "few-rows-one-cta": 1, "few-rows-pair": 2, "row-tile-pair": 3}
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla_decode.so")
 
@@ -79,7 +84,10 @@ def _load() -> ctypes.CDLL:
     L.mla_append_kv.argtypes = [vp, vp, c_i64, vp, c_i64, vp, c_int, c_int, c_int, vp, c_sz, vp]
     L.mla_decode_fwd_append.argtypes = [vp, vp, vp, c_i64, vp, c_i64, vp, c_int, c_int, c_int, c_int, c_f, c_int,
                                         vp, vp, c_int, vp, c_sz, vp, vp, vp]
-    for name in ("mla_get_num_sm_parts", "mla_get_workspace_size", "mla_get_metadata", "mla_decode_fwd",
+    L.mla_set_kernel_variant.argtypes = [c_int]
+    L.mla_get_kernel_variant.argtypes = [c_int]
+    L.mla_get_kernel_variant.restype = c_int
+    for name in ("mla_set_kernel_variant", "mla_get_num_sm_parts", "mla_get_workspace_size", "mla_get_metadata", "mla_decode_fwd",
                  "mla_splitkv_fwd", "mla_combine_fwd", "mla_read_device_status", "mla_append_kv",
                  "mla_decode_fwd_append"):
         getattr(L, name).restype = c_int
@@ -264,6 +272,19 @@ def mla_decode_fwd_append(q, kv_new, kcache, block_table, cache_seqlens, softmax
         raise MlaError("kv_new and q must have the same s_q")
     _check(lib.mla_decode_fwd_append(args[0], _ptr(kv_new), *args[1:]), "mla_decode_fwd_append")
     return out, lse
+
+
+def mla_set_kernel_variant(variant) -> None:
+    """Process-wide split-KV kernel choice: a name of KERNEL_VARIANTS or its number.  Partition
+    counts depend on it: query mla_get_num_sm_parts / mla_get_metadata again afterwards."""
+    v = KERNEL_VARIANTS[variant] if isinstance(variant, str) else int(variant)
+    _check(lib.mla_set_kernel_variant(v), "mla_set_kernel_variant")
+
+
+def mla_get_kernel_variant(rows: int) -> Optional[str]:
+    """Name of the variant a call with s_q * h_q = rows runs now (None if none can)."""
+    v = lib.mla_get_kernel_variant(int(rows))
+    return {n: k for k, n in KERNEL_VARIANTS.items()}.get(v)
 
 
 def mla_read_device_status(workspace: torch.Tensor, stream=None) -> Tuple[int, int]:

@@ -30,7 +30,8 @@ int cuda_fail(cudaError_t e) {
 struct DeviceInfo {
   bool ready = false;
   int sms = 0;
-  int pairs = 0;  // co-resident clusters of 2 split-KV CTAs
+  int pairs = 0;   // co-resident clusters of 2 CTAs of the 128-row-tile kernel
+  int npairs = 0;  // co-resident clusters of 2 CTAs of the few-row pair kernel
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -40,6 +41,16 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // Test hook (mla_test_withhold_q_ready): read by every launch that follows.
 std::atomic<int> g_withhold_q_ready{0};
+// Kernel variant (mla_set_kernel_variant); MLA_KERNEL_AUTO picks by row count.
+std::atomic<int> g_variant{MLA_KERNEL_AUTO};
+
+// The split-KV kernel a call with `rows` = s_q * h_q query rows runs under `variant`
+// (MLA_KERNEL_AUTO resolved), or -1 if that variant cannot take so many rows.
+int kernel_for(int rows, int variant) {
+  if (variant == MLA_KERNEL_AUTO) return rows <= kNarrowMaxRows ? MLA_KERNEL_FEW_ROWS_ONE_CTA : MLA_KERNEL_ROW_TILE_PAIR;
+  if (variant != MLA_KERNEL_ROW_TILE_PAIR && rows > kNarrowMaxRows) return -1;
+  return variant;
+}
 std::atomic<long long> g_wait_cycles{0};
 
 int ensure_encode() {
@@ -100,23 +111,39 @@ int ensure_device(int device) {
       rc = cuda_fail(e);
       break;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * 512);
-    cfg.blockDim = dim3(splitkv_threads());
-    cfg.dynamicSmemBytes = splitkv_smem_bytes();
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, splitkv_kernel_ptr(true), &cfg);
-    if (e != cudaSuccess || clusters <= 0) {
-      (void)cudaGetLastError();
-      clusters = d.sms / 2;  // fall back to the pair count implied by the SM count
+    for (int bf = 0; bf < 2 && rc == MLA_OK; ++bf) {
+      for (int np : {16, 32}) {
+        if ((e = cudaFuncSetAttribute(npair_kernel_ptr(bf == 1, np), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      npair_smem_bytes(np))) != cudaSuccess) {
+          rc = cuda_fail(e);
+          break;
+        }
+      }
     }
+    if (rc != MLA_OK) break;
+    // co-resident clusters of 2 CTAs of a kernel (fallback: the pair count implied by the SM count)
+    auto clusters_of = [&](const void* kernel, int smem, int threads) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2 * 512);
+      cfg.blockDim = dim3(threads);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      cudaError_t ce = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+      if (ce != cudaSuccess || n <= 0) {
+        (void)cudaGetLastError();
+        n = d.sms / 2;
+      }
+      return n;
+    };
+    const int clusters = clusters_of(splitkv_kernel_ptr(true), splitkv_smem_bytes(), splitkv_threads());
+    d.npairs = clusters_of(npair_kernel_ptr(true, 32), npair_smem_bytes(32), splitkv_threads());
     d.pairs = clusters;
     d.ready = true;
   } while (false);
@@ -237,19 +264,28 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
   if ((rc = ensure_encode()) != MLA_OK) return rc;
   const bool bf16 = dtype == MLA_BF16;
   CUtensorMap qrmap, kmap, krmap;
-  const bool narrow = base.rows <= kNarrowMaxRows;
+  const int kernel = kernel_for(base.rows, g_variant.load());
+  if (kernel < 0) return MLA_ERR_UNSUPPORTED;
   if ((rc = encode_3d_k(&kmap, kcache, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf16)) != MLA_OK) return rc;
-  if (!narrow) {  // the pair kernel also takes 32-column boxes of the columns 512..575 of q and of the cache
+  if (kernel != MLA_KERNEL_FEW_ROWS_ONE_CTA) {  // the pair kernels split the columns 512..575 in 32-column boxes
+    if ((rc = encode_3d_k(&krmap, kcache, num_pages, 32, CU_TENSOR_MAP_SWIZZLE_64B, bf16)) != MLA_OK) return rc;
+  }
+  if (kernel == MLA_KERNEL_ROW_TILE_PAIR) {  // ... and the row-tile kernel loads those of q by TMA too
     if ((rc = encode_2d_q(&qrmap, q, static_cast<int64_t>(base.batch) * base.rows, kTileRows, 32,
                           CU_TENSOR_MAP_SWIZZLE_64B, bf16)) != MLA_OK)
       return rc;
-    if ((rc = encode_3d_k(&krmap, kcache, num_pages, 32, CU_TENSOR_MAP_SWIZZLE_64B, bf16)) != MLA_OK) return rc;
   }
   DecodeParams p = base;
   p.block_table = block_table;
   p.block_table_stride = block_table_stride;
   p.num_pages = num_pages;
-  cudaError_t e = narrow ? launch_splitkv_narrow(bf16, q, kmap, p, stream) : launch_splitkv(bf16, q, qrmap, kmap, krmap, p, stream);
+  cudaError_t e;
+  if (kernel == MLA_KERNEL_FEW_ROWS_ONE_CTA)
+    e = launch_splitkv_narrow(bf16, q, kmap, p, stream);
+  else if (kernel == MLA_KERNEL_FEW_ROWS_PAIR)
+    e = launch_splitkv_npair(bf16, q, kmap, krmap, p, stream);
+  else
+    e = launch_splitkv(bf16, q, qrmap, kmap, krmap, p, stream);
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
 }
 
@@ -288,6 +324,17 @@ int mla_last_cuda_error(void) { return g_last_cuda_error; }
 
 int mla_version(void) { return 200; }
 
+int mla_set_kernel_variant(int variant) {
+  if (variant < MLA_KERNEL_AUTO || variant > MLA_KERNEL_ROW_TILE_PAIR) return MLA_ERR_INVALID_ARG;
+  g_variant.store(variant);
+  return MLA_OK;
+}
+
+int mla_get_kernel_variant(int rows) {
+  if (rows < 1 || rows > kMaxRows) return -1;
+  return kernel_for(rows, g_variant.load());
+}
+
 int mla_test_withhold_q_ready(int enable, long long wait_cycles) {
   if (enable != 0 && enable != 1) return MLA_ERR_INVALID_ARG;
   if (wait_cycles < 0) return MLA_ERR_INVALID_ARG;
@@ -302,8 +349,14 @@ int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts) {
   if (rows > kMaxRows) return MLA_ERR_UNSUPPORTED;
   int rc = ensure_device(device);
   if (rc != MLA_OK) return rc;
-  if (rows <= kNarrowMaxRows) {  // one CTA per SM
+  const int kernel = kernel_for(rows, g_variant.load());
+  if (kernel < 0) return MLA_ERR_UNSUPPORTED;
+  if (kernel == MLA_KERNEL_FEW_ROWS_ONE_CTA) {  // one CTA per SM
     *num_sm_parts = g_dev[device].sms > 0 ? g_dev[device].sms : 1;
+    return MLA_OK;
+  }
+  if (kernel == MLA_KERNEL_FEW_ROWS_PAIR) {  // one CTA pair per partition
+    *num_sm_parts = g_dev[device].npairs > 0 ? g_dev[device].npairs : 1;
     return MLA_OK;
   }
   const int m_tiles = (rows + kTileRows - 1) / kTileRows;

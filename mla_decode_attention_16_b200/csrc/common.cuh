@@ -59,4 +59,50 @@ struct DecodeParams {
   int withhold_q_ready;   // test hook: 1 = the first chunk's "Q ready" arrival is never made
 };
 
+// Walks a partition's blocks in order: chunk after chunk (one chunk = the
+// partition's blocks of one request), block after block.
+struct Walk {
+  int br, bk, er, ek;     // the partition's range from the scheduler
+  int req, blk, lo, hi, n;
+  int L;                  // cached tokens of the request
+  int chunk;              // chunk index within the partition
+  bool valid;
+
+  __device__ __forceinline__ void seek(const DecodeParams& p, int from) {
+    for (int r = from; r < p.batch && (r < er || (r == er && ek > 0)); ++r) {
+      L = p.cache_seqlens[r];
+      n = (L + kPage - 1) / kPage;
+      lo = (r == br) ? bk : 0;
+      hi = (r == er) ? ek : n;
+      if (hi > lo) {
+        req = r;
+        blk = lo;
+        valid = true;
+        return;
+      }
+    }
+    valid = false;
+  }
+  __device__ __forceinline__ void init(const DecodeParams& p, const int* meta) {
+    br = meta[0];
+    bk = meta[1];
+    er = meta[2];
+    ek = meta[3];
+    chunk = 0;
+    seek(p, br);
+  }
+  __device__ __forceinline__ void next(const DecodeParams& p) {
+    if (++blk < hi) return;
+    ++chunk;
+    seek(p, req + 1);
+  }
+  // to the first block of the partition's next chunk
+  __device__ __forceinline__ void next_chunk(const DecodeParams& p) {
+    ++chunk;
+    seek(p, req + 1);
+  }
+  __device__ __forceinline__ bool first() const { return blk == lo; }
+  __device__ __forceinline__ bool last() const { return blk == hi - 1; }
+};
+
 }  // namespace mla

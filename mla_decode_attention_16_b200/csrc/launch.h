@@ -22,6 +22,11 @@ int narrow_smem_bytes(int np);
 const void* narrow_kernel_ptr(bool bf16, int np);
 cudaError_t launch_splitkv_narrow(bool bf16, const void* q, const CUtensorMap& kmap, const DecodeParams& p,
                                   cudaStream_t stream);
+// Few-row kernel on a CTA pair (s_q * h_q <= kNarrowMaxRows): one cluster of 2 CTAs per partition.
+int npair_smem_bytes(int np);
+const void* npair_kernel_ptr(bool bf16, int np);
+cudaError_t launch_splitkv_npair(bool bf16, const void* q, const CUtensorMap& kmap, const CUtensorMap& krmap,
+                                 const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_combine(bool bf16, const DecodeParams& p, cudaStream_t stream);
 // Copies kv_new [batch, s_q, 576] into cache positions L_b - s_q + s (programmatic dependent launch).
 cudaError_t launch_append(const void* kv_new, void* kcache, int64_t num_pages, const int32_t* block_table,

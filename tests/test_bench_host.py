@@ -18,8 +18,12 @@ from workloads import WORKLOADS, algorithmic_cost  # noqa: E402
 def test_kernel_choice_by_rows():
     assert bench.kernel_of(1)[0] == "splitkv_narrow_kernel"
     assert bench.kernel_of(32) == ("splitkv_narrow_kernel", "splitkv_narrow.cu")
+    assert bench.kernel_of(16, "few-rows-pair") == ("splitkv_npair_kernel", "splitkv_npair.cu")
     assert bench.kernel_of(33) == ("splitkv_pair_kernel", "splitkv.cu")
     assert bench.kernel_of(1024)[0] == "splitkv_pair_kernel"
+    assert bench.kernel_of(16, "few-rows-one-cta") == ("splitkv_narrow_kernel", "splitkv_narrow.cu")
+    assert bench.kernel_of(16, "row-tile-pair")[0] == "splitkv_pair_kernel"
+    assert bench.variant_of(16) == "few-rows-one-cta" and bench.variant_of(128) == "row-tile-pair"
 
 
 def test_cost_model_by_hand():
@@ -72,5 +76,20 @@ def test_every_bench_workload_has_a_profile_summary():
         if name == "tiny":
             continue
         kernel, _ = bench.kernel_of(WORKLOADS[name].rows)
-        if name in ("memory-bound", "compute-bound"):
-            assert os.path.exists(os.path.join(ROOT, "profiles", f"{kernel}_{name}.md")), name
+        assert os.path.exists(os.path.join(ROOT, "profiles", f"{kernel}_{name}.md")), name
+
+
+def test_sweep_shapes_and_variants():
+    shapes = bench.sweep_shapes()
+    assert (16, 1) in shapes and (128, 8) in shapes and len(shapes) == 16
+    assert all(h * s <= 1024 for h, s in shapes)
+    assert bench.variants_for(32) == ["few-rows-one-cta", "few-rows-pair", "row-tile-pair"]
+    assert bench.variants_for(33) == ["row-tile-pair"]
+
+
+def test_binding_roof_picks_the_slower_roof():
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 100.0}
+    t, b = bench.binding_roof({"bytes": 2e9, "flops": 1e12}, peaks)  # 2 ms of HBM vs 10 ms of tensor
+    assert b == "tensor" and abs(t - 0.01) < 1e-12
+    t, b = bench.binding_roof({"bytes": 2e10, "flops": 1e12}, peaks)
+    assert b == "hbm" and abs(t - 0.02) < 1e-12

@@ -34,14 +34,16 @@ def _hook(lib, enable, cycles):
 
 
 @pytest.mark.parametrize("case", [
-    (3, 1, 16, [700, 64, 2000], False, 1),    # single-CTA kernel (16 rows)
-    (2, 2, 64, [900, 300], True, 2),          # CTA-pair kernel (128 rows)
-], ids=["narrow", "pair"])
+    (3, 1, 16, [700, 64, 2000], False, 1, "few-rows-one-cta"),
+    (3, 1, 16, [700, 64, 2000], False, 1, "few-rows-pair"),
+    (2, 2, 64, [900, 300], True, 2, "row-tile-pair"),
+], ids=lambda c: c[-1])
 def test_withheld_arrival_times_out_and_launch_returns(case):
     import mla_decode_attention_16_b200 as mla
 
-    b, s_q, h_q, lens, causal, seed = case
+    b, s_q, h_q, lens, causal, seed, variant = case
     inp = make_case(b, s_q, h_q, lens, causal=causal, seed=300 + seed)
+    mla.mla_set_kernel_variant(variant)
     _hook(mla.lib, 1, WAIT_CYCLES)
     try:
         t0 = time.perf_counter()
@@ -49,10 +51,15 @@ def test_withheld_arrival_times_out_and_launch_returns(case):
         elapsed = time.perf_counter() - t0
     finally:
         _hook(mla.lib, 0, 0)
+        mla.mla_set_kernel_variant("auto")
     assert flags[0] & 1, f"MLA_DEVERR_TIMEOUT not recorded: {flags}"
     assert elapsed < 30.0
     # the context is intact: the same inputs now run normally and match the oracle
-    out, lse, _, _, flags = run_gpu(inp)
+    mla.mla_set_kernel_variant(variant)
+    try:
+        out, lse, _, _, flags = run_gpu(inp)
+    finally:
+        mla.mla_set_kernel_variant("auto")
     assert flags[0] == 0, flags
     ref_out, ref_lse = oracle.mla_decode_ref(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens,
                                              inp.softmax_scale, inp.causal)

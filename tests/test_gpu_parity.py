@@ -44,6 +44,29 @@ def test_small_cases(case):
     compare(out, lse, ref_out, ref_lse, what=str(case[:4]))
 
 
+FEW_ROWS = [c for c in SMALL if c[1] * c[2] <= 32]
+
+
+@pytest.mark.parametrize("variant", ["few-rows-one-cta", "few-rows-pair", "row-tile-pair"])
+@pytest.mark.parametrize("case", FEW_ROWS, ids=[f"b{c[0]}_sq{c[1]}_h{c[2]}_{c[7]}" for c in FEW_ROWS])
+def test_few_row_cases_every_kernel_variant(variant, case):
+    """Every split-KV kernel that can take s_q * h_q <= 32 rows gives the oracle's result."""
+    import mla_decode_attention_16_b200 as mla
+
+    b, s_q, h_q, lens, dtype, causal, parts, seed = case
+    inp = make_case(b, s_q, h_q, lens, dtype=dtype, causal=causal, seed=seed, extra_poison_pages=3, table_pad=2)
+    mla.mla_set_kernel_variant(variant)
+    try:
+        assert mla.mla_get_kernel_variant(s_q * h_q) == variant
+        out, lse, meta, ns, flags = run_gpu(inp, parts)
+    finally:
+        mla.mla_set_kernel_variant("auto")
+    assert flags[0] == 0, flags
+    ref_out, ref_lse = oracle.mla_decode_ref(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens,
+                                             inp.softmax_scale, inp.causal)
+    compare(out, lse, ref_out, ref_lse, what=f"{variant} {case[:4]}")
+
+
 def test_tiny_workload():
     inp = make_workload("tiny")
     out, lse, _, _, flags = run_gpu(inp)
