@@ -19,6 +19,11 @@ sched_ref.tile_schedule_ref
 append_ref.append_kv_ref / append_ref.decode_with_append_ref
     the new tokens' rows written into their page slots (the step before a
     decode), and "append, then decode".
+fp8_ref.mla_decode_fp8_ref / fp8_ref.append_kv_fp8_ref
+    the FP8 (e5m2) cache variant: the query cast to e5m2, the cache's e5m2
+    values as K and V, the plain decode on those values; the append that casts
+    the new rows to e5m2 (``e5m2_quantize`` / ``e5m2_encode`` / ``e5m2_decode``:
+    the format and its round-to-nearest-even cast).
 
 Sources (pages, by title and section)
 -------------------------------------
@@ -34,9 +39,12 @@ Sources (pages, by title and section)
   结果融合 (merge the chunk outputs with dynamic weights).
 * "FlashAttention终极指南" (cnnetsun.cn): ``cache_seqlens`` / ``causal`` /
   ``return_softmax_lse`` conventions of a KV-cache attention call.
+* "云上AI推理新突破：FlashMLA赋能DeepSeek-V2-Lite提速16%", section 3. 动态精度缩放,
+  and "DeepSeek开源FlashMLA全解析", section 1.2 计算模式创新: Q.K^T from float8_e5m2
+  operands, softmax and P.V back at FP16 precision.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-(``tests/append_pins.py`` for the append)
+(``tests/append_pins.py`` for the append, ``tests/fp8_pins.py`` for the FP8 variant)
 (closed forms, invariants, brute force, an independent library special case)
 and ``tests/test_oracle_mutants.py`` (planted mistakes must fail a pin).
 """
@@ -52,3 +60,10 @@ from .mla_ref import (  # noqa: F401
 )
 from .sched_ref import FIXED_OVERHEAD_BLOCKS, tile_schedule_ref  # noqa: F401
 from .append_ref import append_kv_ref, decode_with_append_ref  # noqa: F401
+from .fp8_ref import (  # noqa: F401
+    append_kv_fp8_ref,
+    e5m2_decode,
+    e5m2_encode,
+    e5m2_quantize,
+    mla_decode_fp8_ref,
+)

@@ -13,9 +13,11 @@ import types
 import pytest
 
 import oracle.append_ref as app
+import oracle.fp8_ref as fp8
 import oracle.mla_ref as ref
 import oracle.sched_ref as sched
 from append_pins import ALL_APPEND_PINS
+from fp8_pins import ALL_FP8_PINS
 from oracle_pins import ALL_PINS
 from sched_pins import ALL_SCHED_PINS
 
@@ -71,6 +73,23 @@ APPEND_MUTANTS = {
     "short request wraps around": ("            if j < 0:\n                continue\n", ""),
 }
 
+FP8_MUTANTS = {
+    "ties round up": ("q = torch.round(safe / spacing) * spacing", "q = torch.floor(safe / spacing + 0.5) * spacing"),
+    "truncation": ("q = torch.round(safe / spacing) * spacing", "q = torch.floor(safe / spacing) * spacing"),
+    "exponent bias 16": ("E5M2_BIAS = 15", "E5M2_BIAS = 16"),
+    "three mantissa bits": ("E5M2_MANT_BITS = 2", "E5M2_MANT_BITS = 3"),
+    "no subnormal floor": ("e = (k.to(torch.int64) - 1).clamp(min=E5M2_MIN_NORMAL_EXP)", "e = k.to(torch.int64) - 1"),
+    "binade off by one": ("e = (k.to(torch.int64) - 1).clamp(min=E5M2_MIN_NORMAL_EXP)",
+                          "e = k.to(torch.int64).clamp(min=E5M2_MIN_NORMAL_EXP)"),
+    "overflow not saturated": ("q = torch.clamp(q, max=E5M2_MAX)", "q = q"),
+    "subnormals one binade low": ("return sign * (m / 4.0) * 2.0 ** E5M2_MIN_NORMAL_EXP",
+                                  "return sign * (m / 4.0) * 2.0 ** (E5M2_MIN_NORMAL_EXP - 1)"),
+    "mantissa bits swapped": ("m = code & 0x3", "m = ((code & 1) << 1) | ((code >> 1) & 1)"),
+    "query not cast": ("q8 = e5m2_quantize(q.to(_F64))", "q8 = q.to(_F64)"),
+    "append stores truncated bytes": ("e5m2_encode(kv_new.to(_F64)))", "kv_new.to(torch.uint8))"),
+    "sign dropped": ("out = torch.where(finite_nz, torch.copysign(q, x), x)", "out = torch.where(finite_nz, q, x)"),
+}
+
 
 def _mutant(module: types.ModuleType, edits) -> types.ModuleType:
     """Copy of ``module`` with each (old, new) text substitution applied."""
@@ -118,3 +137,9 @@ def test_append_mutant_is_caught(name):
 def test_sched_mutant_is_caught(name):
     mod = _mutant(sched, SCHED_MUTANTS[name])
     assert _caught(ALL_SCHED_PINS, mod), f"mutant '{name}' passed every pin"
+
+
+@pytest.mark.parametrize("name", sorted(FP8_MUTANTS))
+def test_fp8_mutant_is_caught(name):
+    mod = _mutant(fp8, FP8_MUTANTS[name])
+    assert _caught(ALL_FP8_PINS, mod), f"mutant '{name}' passed every pin"
