@@ -5,10 +5,12 @@ A step is one pass of the whole hot path over one batch: the tile scheduler
 kernel), inputs resident in HBM.  The headline workload is the memory-bound
 decode batch (64 requests x 4096 cached tokens, h_q 16, s_q 1, bf16); a
 default run adds, under "per_workload", the same measurements for the three
-workloads with h_q * s_q >= 128 (compute-bound, varlen-mtp, long-fp16; at most
---companion-steps timed steps each).  Pick one workload with --workload.
-Throughput uses the pages' cost model: bytes = 576*2*sum(L) + q + out + lse,
-FLOPs = 2*h_q*s_q*(576+512)*sum(L).
+workloads with h_q * s_q >= 128 (compute-bound, varlen-mtp, long-fp16) and for
+the memory-bound batch over an e5m2 cache (memory-bound-fp8), at most
+--companion-steps timed steps each.  Pick one workload with --workload.
+Throughput uses the pages' cost model: bytes = 576*e*sum(L) + q + out + lse
+(e = 2 bytes per cached value, 1 for the e5m2 cache), FLOPs =
+2*h_q*s_q*(576+512)*sum(L).
 
 Timing: W warm-up steps, then exactly K steps between CUDA events on the
 launching stream, with a barrier and a synchronize on both sides; two resident
@@ -168,9 +170,25 @@ def variant_of(rows: int, variant: str = "auto") -> str:
     return "few-rows-one-cta" if rows <= 32 else "row-tile-pair"
 
 
-def kernel_of(rows: int, variant: str = "auto"):
-    """(name, source file) of the split-KV kernel the library runs for s_q * h_q = rows."""
-    return KERNELS[variant_of(rows, variant)]
+FP8_KERNEL = ("splitkv_fp8_kernel", "splitkv_fp8.cu")
+
+
+def kernel_of(rows: int, variant: str = "auto", kv_fp8: bool = False):
+    """(name, source file) of the split-KV kernel the library runs for s_q * h_q = rows (one kernel
+    takes every row count over an e5m2 cache)."""
+    return FP8_KERNEL if kv_fp8 else KERNELS[variant_of(rows, variant)]
+
+
+def cost_of(inp, lens):
+    """The pages' cost model for these requests of a workload (1 byte per value of an e5m2 cache)."""
+    return algorithmic_cost(lens, inp.s_q, inp.h_q, kv_elem_bytes=inp.kcache.element_size())
+
+
+def oracle_fn(inp):
+    """The CPU oracle's decode for this workload's cache type."""
+    import oracle
+
+    return oracle.mla_decode_fp8_ref if inp.kcache.dtype == torch.uint8 else oracle.mla_decode_ref
 
 
 def profile_traffic(name: str, kernel: str, source: str):
@@ -197,14 +215,13 @@ def oracle_sample(inp, budget_s: float, min_s: float = 3.0):
     seconds have passed (so a workload the oracle finishes quickly is still timed over a few
     seconds); it stops early once budget_s is reached.
     """
-    import oracle
-
+    decode = oracle_fn(inp)
     done, t0, passes = [], time.perf_counter(), 0
     floor = min(min_s, budget_s)
     while True:
         for r in range(inp.batch):
-            oracle.mla_decode_ref(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens, inp.softmax_scale,
-                                  inp.causal, requests=[r])
+            decode(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens, inp.softmax_scale, inp.causal,
+                   requests=[r])
             done.append(r)
             if time.perf_counter() - t0 >= budget_s:
                 return time.perf_counter() - t0, done, passes
@@ -216,7 +233,7 @@ def oracle_sample(inp, budget_s: float, min_s: float = 3.0):
 def cpu_baseline(inp, name: str, unit: str, budget_s: float):
     secs, reqs, passes = oracle_sample(inp, budget_s)
     lens = [int(inp.cache_seqlens[r]) for r in reqs]
-    cost = algorithmic_cost(lens, inp.s_q, inp.h_q)
+    cost = cost_of(inp, lens)
     what = (f"{passes} full pass(es) over the {inp.batch} requests" if len(reqs) == passes * inp.batch
             else f"{len(reqs)} request(s) in order")
     return {"value": throughput(cost, secs, unit), "unit": unit, "cores": torch.get_num_threads(),
@@ -237,7 +254,7 @@ def run_reference(args, name: str):
     for _ in range(args.steps):
         secs, reqs, _ = oracle_sample(inp, per_step, per_step)
         lens = [int(inp.cache_seqlens[r]) for r in reqs]
-        vals.append(throughput(algorithmic_cost(lens, inp.s_q, inp.h_q), secs, unit))
+        vals.append(throughput(cost_of(inp, lens), secs, unit))
         secs_tot += secs
     value = statistics.median(vals)
     w = WORKLOADS[name]
@@ -286,9 +303,11 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
     calls in the same order; rank 0 gets the result dict, the others None."""
     import mla_decode_attention_16_b200 as mla
 
+    w = WORKLOADS[name]
+    if w.kv_fp8:
+        variant = "auto"  # the e5m2-cache kernel has no variants
     mla.mla_set_kernel_variant(variant)
     unit = unit_of(name)
-    w = WORKLOADS[name]
     if rank == 0:
         inp = make_workload(name)
     else:
@@ -296,9 +315,9 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
         g = torch.Generator().manual_seed(shard_seed(w.seed, rank))  # same shapes and length law
         lens = wl.draw_seqlens(w, g)
         inp = wl.make_case(w.batch, w.s_q, w.h_q, lens, dtype=w.dtype, std=w.std, causal=w.causal,
-                           seed=shard_seed(w.seed, rank) + 1)
+                           seed=shard_seed(w.seed, rank) + 1, kv_fp8=w.kv_fp8)
     lens = [int(x) for x in inp.cache_seqlens.tolist()]
-    cost = algorithmic_cost(lens, inp.s_q, inp.h_q)
+    cost = cost_of(inp, lens)
 
     b, s_q, h_q = inp.batch, inp.s_q, inp.h_q
     rows = s_q * h_q
@@ -306,7 +325,7 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
     caches = [inp.kcache.to(dev), inp.kcache.to(dev)]
     bt = inp.block_table.to(dev)
     sl = inp.cache_seqlens.to(dev)
-    parts = mla.mla_get_num_sm_parts(rows, dev.index)
+    parts = mla.mla_get_num_sm_parts(rows, dev.index, kv_fp8=w.kv_fp8)
     meta = torch.empty(parts, 8, dtype=torch.int32, device=dev)
     ns = torch.empty(b + 1, dtype=torch.int32, device=dev)
     ws = mla.alloc_workspace(b, rows, parts, dev)
@@ -438,17 +457,17 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
         achieved = cost["flops"] / kern_s / 1e12
         peak = float(peaks["bf16_tflops"])  # fp16 dense tensor rate equals bf16 on this part
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
-    kname, ksrc = kernel_of(rows, variant)
+    kname, ksrc = kernel_of(rows, variant, w.kv_fp8)
     roof["traffic"] = profile_traffic(name, kname, ksrc)
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["kernel"] = kname
-    roof["variant"] = variant_of(rows, variant)
+    roof["variant"] = "fp8-cache" if w.kv_fp8 else variant_of(rows, variant)
     roof["kernel_us"] = kern_s * 1e6
     roof["algorithmic_per_launch"] = cost["bytes"] if unit == "GB/s" else cost["flops"]
     res = {
         "value": value, "unit": unit, "steps": steps, "warmup": warmup,
         "ms_per_step": 1000.0 * elapsed_max / steps,
-        "dtype": "bf16" if q.dtype == torch.bfloat16 else "fp16",
+        "dtype": ("e5m2 q.k, fp16 p.v, " if w.kv_fp8 else "") + ("bf16" if q.dtype == torch.bfloat16 else "fp16"),
         "config": workload_config(name, world),
         "tflops": cost["flops"] / (elapsed_max / steps) / 1e12 * world,
         "gbps": cost["bytes"] / (elapsed_max / steps) / 1e9 * world,
@@ -548,8 +567,9 @@ def run_sweep(args):
     return 0
 
 
-# workloads whose numbers join the headline line of a default run (the pages' h_q * s_q >= 128 configs)
-COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16"]
+# workloads whose numbers join the headline line of a default run: the pages' h_q * s_q >= 128
+# configs, and the headline batch over the e5m2 cache
+COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16", "memory-bound-fp8"]
 
 
 def run_gpu(args, name: str, companions=()):

@@ -69,6 +69,22 @@ typedef enum {
 
 typedef enum { MLA_BF16 = 0, MLA_FP16 = 1 } mla_dtype;
 
+/*
+ * FP8 cache ("云上AI推理新突破：FlashMLA赋能DeepSeek-V2-Lite提速16%", section
+ * 3. 动态精度缩放; "DeepSeek开源FlashMLA全解析", section 1.2 计算模式创新): OR-ed
+ * into the dtype argument of the decode, split-KV, combine and append calls
+ * (MLA_BF16 | MLA_KV_FP8_E5M2, MLA_FP16 | MLA_KV_FP8_E5M2), it says that
+ * kcache holds float8 e5m2 values, one byte each ([num_pages, 64, 1, 576]
+ * bytes, 16-B aligned); q, kv_new and out keep the base dtype.  The decode
+ * casts q to e5m2 (round to nearest even; finite values beyond 57344
+ * saturate), forms q.K from the 8-bit values with fp32 accumulation, runs the
+ * softmax in fp32, rounds P to fp16 and multiplies it by V widened to fp16
+ * (exact).  The append casts each new value to e5m2 the same way.  Kernel
+ * variants (mla_set_kernel_variant) do not apply: one kernel takes every row
+ * count, in tiles of 32 query rows.
+ */
+#define MLA_KV_FP8_E5M2 0x100
+
 /* Human-readable name of a status code (static string). */
 const char* mla_status_string(int status);
 
@@ -133,6 +149,15 @@ int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts);
 int mla_get_workspace_size(int batch, int rows, int num_sm_parts, size_t* bytes);
 
 /*
+ * mla_get_num_sm_parts for a given dtype argument: with MLA_KV_FP8_E5M2 set,
+ * the e5m2-cache kernel runs one CTA per (partition, tile of 32 query rows)
+ * and SM, so num_sm_parts = SMs / ceil(rows / 32) (at least 1); without it,
+ * the same as mla_get_num_sm_parts.  Any num_sm_parts >= 1 gives correct
+ * results; this one fills the GPU once.
+ */
+int mla_get_num_sm_parts_dtype(int device, int rows, int dtype, int* num_sm_parts);
+
+/*
  * Tile scheduler ("FlashMLA: 高性能GPU注意力机制计算库", section 6. SM资源调度优化).
  *   cache_seqlens        device int32 [batch]: cached tokens per request (>= 0)
  *   batch                1 .. 16384
@@ -174,7 +199,8 @@ int mla_get_metadata(const int32_t* cache_seqlens, int batch, int rows, int num_
  *   block_table_stride  elements between rows of block_table (>= 1)
  *   cache_seqlens     device int32 [batch], the same values given to mla_get_metadata
  *   batch, s_q, h_q   s_q * h_q in [1, 1024]
- *   dtype             MLA_BF16 or MLA_FP16 (q, kcache and out share it)
+ *   dtype             MLA_BF16 or MLA_FP16 (q, kcache and out share it), optionally
+ *                     | MLA_KV_FP8_E5M2 (kcache holds e5m2 bytes; see above)
  *   softmax_scale     multiplies q.k (finite)
  *   causal            0 or 1 (see the header comment)
  *   tile_sched_metadata, num_splits, num_sm_parts   from mla_get_metadata

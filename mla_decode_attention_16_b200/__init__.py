@@ -13,6 +13,10 @@ Typical use::
     ws = alloc_workspace(batch, s_q * h_q, parts)
     out, lse = mla_decode_fwd(q, kcache, block_table, cache_seqlens, 576 ** -0.5, False,
                               meta, num_splits, ws)
+
+A cache of dtype ``torch.uint8`` or ``torch.float8_e5m2`` holds e5m2 values (one byte each); the
+call then passes the base dtype of q with ``KV_FP8_E5M2`` (include/mla_decode.h), and partition
+counts come from ``mla_get_num_sm_parts(rows, kv_fp8=True)``.
 """
 
 from __future__ import annotations
@@ -29,6 +33,7 @@ __all__ = [
     "library_path",
     "mla_version",
     "mla_get_num_sm_parts",
+    "KV_FP8_E5M2",
     "mla_get_workspace_size",
     "alloc_workspace",
     "mla_get_metadata",
@@ -52,6 +57,8 @@ HEAD_DIM_V = 512
 PAGE_SIZE = 64
 META_INTS = 8
 _DTYPES = {torch.bfloat16: 0, torch.float16: 1}
+KV_FP8_E5M2 = 0x100  # OR-ed into the dtype code: the cache holds e5m2 bytes
+_FP8_CACHE = (torch.uint8, torch.float8_e5m2)
 # split-KV kernel variants (include/mla_decode.h, MLA_KERNEL_*)
 KERNEL_VARIANTS = {"auto": 0, "few-rows-one-cta": 1, "few-rows-pair": 2, "row-tile-pair": 3}
 
@@ -74,6 +81,7 @@ def _load() -> ctypes.CDLL:
     L.mla_last_cuda_error.restype = c_int
     L.mla_version.restype = c_int
     L.mla_get_num_sm_parts.argtypes = [c_int, c_int, ctypes.POINTER(c_int)]
+    L.mla_get_num_sm_parts_dtype.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_int)]
     L.mla_get_workspace_size.argtypes = [c_int, c_int, c_int, ctypes.POINTER(c_sz)]
     L.mla_get_metadata.argtypes = [vp, c_int, c_int, c_int, vp, vp, vp]
     fwd = [vp, vp, c_i64, vp, c_i64, vp, c_int, c_int, c_int, c_int, c_f, c_int, vp, vp, c_int, vp, c_sz, vp, vp, vp]
@@ -87,7 +95,7 @@ def _load() -> ctypes.CDLL:
     L.mla_set_kernel_variant.argtypes = [c_int]
     L.mla_get_kernel_variant.argtypes = [c_int]
     L.mla_get_kernel_variant.restype = c_int
-    for name in ("mla_set_kernel_variant", "mla_get_num_sm_parts", "mla_get_workspace_size", "mla_get_metadata", "mla_decode_fwd",
+    for name in ("mla_set_kernel_variant", "mla_get_num_sm_parts", "mla_get_num_sm_parts_dtype", "mla_get_workspace_size", "mla_get_metadata", "mla_decode_fwd",
                  "mla_splitkv_fwd", "mla_combine_fwd", "mla_read_device_status", "mla_append_kv",
                  "mla_decode_fwd_append"):
         getattr(L, name).restype = c_int
@@ -119,11 +127,21 @@ def mla_version() -> int:
     return lib.mla_version()
 
 
-def mla_get_num_sm_parts(rows: int, device: Optional[int] = None) -> int:
+def mla_get_num_sm_parts(rows: int, device: Optional[int] = None, kv_fp8: bool = False) -> int:
+    """Scheduler partitions for s_q * h_q = rows (kv_fp8: for an e5m2 cache)."""
     dev = torch.cuda.current_device() if device is None else int(device)
     out = ctypes.c_int(0)
-    _check(lib.mla_get_num_sm_parts(dev, int(rows), ctypes.byref(out)), "mla_get_num_sm_parts")
+    if kv_fp8:
+        _check(lib.mla_get_num_sm_parts_dtype(dev, int(rows), KV_FP8_E5M2, ctypes.byref(out)),
+               "mla_get_num_sm_parts_dtype")
+    else:
+        _check(lib.mla_get_num_sm_parts(dev, int(rows), ctypes.byref(out)), "mla_get_num_sm_parts")
     return out.value
+
+
+def _cache_code(kcache: torch.Tensor, base: torch.dtype) -> int:
+    """dtype code of a call whose 16-bit tensors are `base` and whose cache is kcache."""
+    return _DTYPES[base] | (KV_FP8_E5M2 if kcache.dtype in _FP8_CACHE else 0)
 
 
 def mla_get_workspace_size(batch: int, rows: int, num_sm_parts: int) -> int:
@@ -180,7 +198,7 @@ def _fwd_args(q, kcache, block_table, cache_seqlens, softmax_scale, causal, tile
     b, s_q, h_q, dk = q.shape
     if dk != HEAD_DIM_K:
         raise MlaError(f"q last dim must be {HEAD_DIM_K}")
-    _need(kcache, "kcache", q.dtype, 4)
+    _need(kcache, "kcache", None if kcache.dtype in _FP8_CACHE else q.dtype, 4)
     if tuple(kcache.shape[1:]) != (PAGE_SIZE, 1, HEAD_DIM_K):
         raise MlaError(f"kcache must be [pages, {PAGE_SIZE}, 1, {HEAD_DIM_K}], got {tuple(kcache.shape)}")
     _need(block_table, "block_table", torch.int32, 2)
@@ -203,7 +221,7 @@ def _fwd_args(q, kcache, block_table, cache_seqlens, softmax_scale, causal, tile
     if tuple(out.shape) != (b, s_q, h_q, HEAD_DIM_V) or tuple(lse.shape) != (b, h_q, s_q):
         raise MlaError("out / lse shapes do not match q")
     args = (_ptr(q), _ptr(kcache), kcache.shape[0], _ptr(block_table), block_table.stride(0), _ptr(cache_seqlens),
-            b, s_q, h_q, _DTYPES[q.dtype], float(softmax_scale), 1 if causal else 0, _ptr(tile_sched_metadata),
+            b, s_q, h_q, _cache_code(kcache, q.dtype), float(softmax_scale), 1 if causal else 0, _ptr(tile_sched_metadata),
             _ptr(num_splits), parts, _ptr(workspace), workspace.numel(), _ptr(out), _ptr(lse),
             _stream(stream, q.device))
     return args, out, lse
@@ -239,7 +257,9 @@ def mla_combine_fwd(cache_seqlens, s_q, h_q, dtype, num_splits, num_sm_parts, wo
 
 
 def _check_kv_new(kv_new, kcache, block_table):
-    _need(kv_new, "kv_new", kcache.dtype, 3)
+    _need(kv_new, "kv_new", None if kcache.dtype in _FP8_CACHE else kcache.dtype, 3)
+    if kv_new.dtype not in _DTYPES:
+        raise MlaError(f"kv_new must be bf16 or fp16, got {kv_new.dtype}")
     if kv_new.shape[0] != block_table.shape[0] or kv_new.shape[2] != HEAD_DIM_K:
         raise MlaError(f"kv_new must be [batch, s_q, {HEAD_DIM_K}], got {tuple(kv_new.shape)}")
 
@@ -248,15 +268,16 @@ def mla_append_kv(kv_new, kcache, block_table, cache_seqlens, workspace, stream=
     """Write kv_new [b, s_q, 576] into the cache at positions L_b - s_q + s (in place); see
     include/mla_decode.h.  Returns kcache."""
     _need(kcache, "kcache", dim=4)
-    if kcache.dtype not in _DTYPES:
-        raise MlaError(f"kcache must be bf16 or fp16, got {kcache.dtype}")
+    if kcache.dtype not in _DTYPES and kcache.dtype not in _FP8_CACHE:
+        raise MlaError(f"kcache must be bf16, fp16 or e5m2 bytes, got {kcache.dtype}")
     _need(block_table, "block_table", torch.int32, 2)
     _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8, 1)
     _check_kv_new(kv_new, kcache, block_table)
     b, s_q, _ = kv_new.shape
     _check(lib.mla_append_kv(_ptr(kv_new), _ptr(kcache), kcache.shape[0], _ptr(block_table), block_table.stride(0),
-                             _ptr(cache_seqlens), b, s_q, _DTYPES[kcache.dtype], _ptr(workspace), workspace.numel(),
+                             _ptr(cache_seqlens), b, s_q, _cache_code(kcache, kv_new.dtype), _ptr(workspace),
+                             workspace.numel(),
                              _stream(stream, kcache.device)), "mla_append_kv")
     return kcache
 
@@ -270,6 +291,8 @@ def mla_decode_fwd_append(q, kv_new, kcache, block_table, cache_seqlens, softmax
     _check_kv_new(kv_new, kcache, block_table)
     if kv_new.shape[1] != q.shape[1]:
         raise MlaError("kv_new and q must have the same s_q")
+    if kv_new.dtype != q.dtype:
+        raise MlaError("kv_new and q must have the same dtype")
     _check(lib.mla_decode_fwd_append(args[0], _ptr(kv_new), *args[1:]), "mla_decode_fwd_append")
     return out, lse
 

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmla_decode.so")
-SOURCES = ["api.cu", "metadata.cu", "splitkv.cu", "splitkv_narrow.cu", "splitkv_npair.cu", "combine.cu", "append.cu", "static_ws.cu"]
+SOURCES = ["api.cu", "metadata.cu", "splitkv.cu", "splitkv_narrow.cu", "splitkv_npair.cu", "splitkv_fp8.cu", "combine.cu", "append.cu", "static_ws.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -36,7 +36,8 @@ def _nvcc() -> str:
 
 def _inputs():
     files = [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE)]
-    return [f for f in files if f.endswith((".cu", ".cuh", ".h"))]
+    # build.py itself: the source list and flags live here
+    return [f for f in files if f.endswith((".cu", ".cuh", ".h"))] + [os.path.abspath(__file__)]
 
 
 def needs_build() -> bool:

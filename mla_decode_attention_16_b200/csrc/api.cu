@@ -106,6 +106,16 @@ int ensure_device(int device) {
       }
     }
     if (rc != MLA_OK) break;
+    for (int bf = 0; bf < 2 && rc == MLA_OK; ++bf) {
+      for (int np : {16, 32}) {
+        if ((e = cudaFuncSetAttribute(fp8_kernel_ptr(bf == 1, np), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      fp8_smem_bytes(np))) != cudaSuccess) {
+          rc = cuda_fail(e);
+          break;
+        }
+      }
+    }
+    if (rc != MLA_OK) break;
     if ((e = cudaFuncSetAttribute(metadata_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   metadata_smem_bytes(kMaxBatch, kMaxParts))) != cudaSuccess) {
       rc = cuda_fail(e);
@@ -202,6 +212,30 @@ int encode_3d_k(CUtensorMap* map, const void* kc, int64_t num_pages, int box_col
   return MLA_OK;
 }
 
+// Box of box_cols columns x one 64-token page of an e5m2 cache viewed as [pages, 64, 576] bytes.
+int encode_3d_k8(CUtensorMap* map, const void* kc, int64_t num_pages, int box_cols, CUtensorMapSwizzle swizzle) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDK), static_cast<cuuint64_t>(kPage),
+                              static_cast<cuuint64_t>(num_pages)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDK), static_cast<cuuint64_t>(kDK) * kPage};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kPage), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kc), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}
+
+bool valid_dtype(int dtype) {
+  const int base = dtype & ~MLA_KV_FP8_E5M2;
+  return base == MLA_BF16 || base == MLA_FP16;
+}
+bool is_bf16(int dtype) { return (dtype & ~MLA_KV_FP8_E5M2) == MLA_BF16; }
+bool is_kv8(int dtype) { return (dtype & MLA_KV_FP8_E5M2) != 0; }
+
 // Shared checks + parameter packing of the forward calls.
 int prepare(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int dtype, int causal,
             const int32_t* meta, const int32_t* num_splits, int num_sm_parts, void* workspace,
@@ -211,7 +245,7 @@ int prepare(const int32_t* cache_seqlens, int batch, int s_q, int h_q, int dtype
   if (batch > kMaxBatch) return MLA_ERR_UNSUPPORTED;
   int rc = check_rows(s_q, h_q);
   if (rc != MLA_OK) return rc;
-  if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return MLA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (!aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_INVALID_ARG;
@@ -262,8 +296,19 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
   if (rc != MLA_OK) return rc;
   if ((rc = ensure_device(dev)) != MLA_OK) return rc;
   if ((rc = ensure_encode()) != MLA_OK) return rc;
-  const bool bf16 = dtype == MLA_BF16;
+  const bool bf16 = is_bf16(dtype);
   CUtensorMap qrmap, kmap, krmap;
+  DecodeParams p = base;
+  p.block_table = block_table;
+  p.block_table_stride = block_table_stride;
+  p.num_pages = num_pages;
+  cudaError_t e;
+  if (is_kv8(dtype)) {  // e5m2 cache: 128-column boxes (128-byte swizzle) + the 64 columns 512..575
+    if ((rc = encode_3d_k8(&kmap, kcache, num_pages, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK) return rc;
+    if ((rc = encode_3d_k8(&krmap, kcache, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK) return rc;
+    e = launch_splitkv_fp8(bf16, q, kmap, krmap, p, stream);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e);
+  }
   const int kernel = kernel_for(base.rows, g_variant.load());
   if (kernel < 0) return MLA_ERR_UNSUPPORTED;
   if ((rc = encode_3d_k(&kmap, kcache, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf16)) != MLA_OK) return rc;
@@ -275,11 +320,6 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
                           CU_TENSOR_MAP_SWIZZLE_64B, bf16)) != MLA_OK)
       return rc;
   }
-  DecodeParams p = base;
-  p.block_table = block_table;
-  p.block_table_stride = block_table_stride;
-  p.num_pages = num_pages;
-  cudaError_t e;
   if (kernel == MLA_KERNEL_FEW_ROWS_ONE_CTA)
     e = launch_splitkv_narrow(bf16, q, kmap, p, stream);
   else if (kernel == MLA_KERNEL_FEW_ROWS_PAIR)
@@ -322,7 +362,7 @@ const char* mla_status_string(int status) {
 
 int mla_last_cuda_error(void) { return g_last_cuda_error; }
 
-int mla_version(void) { return 200; }
+int mla_version(void) { return 210; }
 
 int mla_set_kernel_variant(int variant) {
   if (variant < MLA_KERNEL_AUTO || variant > MLA_KERNEL_ROW_TILE_PAIR) return MLA_ERR_INVALID_ARG;
@@ -361,6 +401,18 @@ int mla_get_num_sm_parts(int device, int rows, int* num_sm_parts) {
   }
   const int m_tiles = (rows + kTileRows - 1) / kTileRows;
   const int parts = g_dev[device].pairs / m_tiles;
+  *num_sm_parts = parts > 0 ? parts : 1;
+  return MLA_OK;
+}
+
+int mla_get_num_sm_parts_dtype(int device, int rows, int dtype, int* num_sm_parts) {
+  if (!valid_dtype(dtype)) return MLA_ERR_INVALID_ARG;
+  if (!is_kv8(dtype)) return mla_get_num_sm_parts(device, rows, num_sm_parts);
+  if (!num_sm_parts || rows < 1) return MLA_ERR_INVALID_ARG;
+  if (rows > kMaxRows) return MLA_ERR_UNSUPPORTED;
+  int rc = ensure_device(device);
+  if (rc != MLA_OK) return rc;
+  const int parts = g_dev[device].sms / fp8_row_tiles(rows);  // one CTA per (partition, 32-row tile) per SM
   *num_sm_parts = parts > 0 ? parts : 1;
   return MLA_OK;
 }
@@ -407,7 +459,7 @@ int mla_combine_fwd(const int32_t* cache_seqlens, int batch, int s_q, int h_q, i
   int rc = prepare(cache_seqlens, batch, s_q, h_q, dtype, 0, num_splits, num_splits, num_sm_parts, workspace,
                    workspace_bytes, out, lse, 1.0f, &p);
   if (rc != MLA_OK) return rc;
-  cudaError_t e = launch_combine(dtype == MLA_BF16, p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_combine(is_bf16(dtype), p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
 }
 
@@ -422,7 +474,7 @@ int mla_decode_fwd(const void* q, const void* kcache, int64_t num_pages, const i
   if (rc != MLA_OK) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((rc = splitkv_impl(q, kcache, num_pages, block_table, block_table_stride, p, dtype, st)) != MLA_OK) return rc;
-  cudaError_t e = launch_combine(dtype == MLA_BF16, p, st);
+  cudaError_t e = launch_combine(is_bf16(dtype), p, st);
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
 }
 
@@ -433,12 +485,16 @@ int mla_append_kv(const void* kv_new, void* kcache, int64_t num_pages, const int
   if (batch < 1 || s_q < 1 || num_pages < 1 || block_table_stride < 1) return MLA_ERR_INVALID_ARG;
   if (batch > kMaxBatch || s_q > kMaxRows) return MLA_ERR_UNSUPPORTED;
   if (num_pages > (int64_t(1) << 31) - 1) return MLA_ERR_UNSUPPORTED;
-  if (dtype != MLA_BF16 && dtype != MLA_FP16) return MLA_ERR_INVALID_ARG;
+  if (!valid_dtype(dtype)) return MLA_ERR_INVALID_ARG;
   if (!aligned16(kv_new) || !aligned16(kcache) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return MLA_ERR_INVALID_ARG;
   if (workspace_bytes < kWsHeader) return MLA_ERR_WORKSPACE;
-  cudaError_t e = launch_append(kv_new, kcache, num_pages, block_table, block_table_stride, cache_seqlens, batch,
-                                s_q, static_cast<int*>(workspace), static_cast<cudaStream_t>(stream));
+  cudaError_t e = is_kv8(dtype)
+                      ? launch_append_fp8(is_bf16(dtype), kv_new, kcache, num_pages, block_table, block_table_stride,
+                                          cache_seqlens, batch, s_q, static_cast<int*>(workspace),
+                                          static_cast<cudaStream_t>(stream))
+                      : launch_append(kv_new, kcache, num_pages, block_table, block_table_stride, cache_seqlens,
+                                      batch, s_q, static_cast<int*>(workspace), static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MLA_OK : cuda_fail(e);
 }
 

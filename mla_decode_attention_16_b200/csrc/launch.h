@@ -27,11 +27,22 @@ int npair_smem_bytes(int np);
 const void* npair_kernel_ptr(bool bf16, int np);
 cudaError_t launch_splitkv_npair(bool bf16, const void* q, const CUtensorMap& kmap, const CUtensorMap& krmap,
                                  const DecodeParams& p, cudaStream_t stream);
+// Split-KV kernel over an e5m2 cache, any row count: one CTA per (partition, 32-row tile).
+// kmap: 128-column boxes (128-byte swizzle); krmap: the 64 columns 512..575 (64-byte swizzle).
+int fp8_row_tiles(int rows);
+int fp8_smem_bytes(int np);
+const void* fp8_kernel_ptr(bool bf16, int np);
+cudaError_t launch_splitkv_fp8(bool bf16, const void* q, const CUtensorMap& kmap, const CUtensorMap& krmap,
+                               const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_combine(bool bf16, const DecodeParams& p, cudaStream_t stream);
 // Copies kv_new [batch, s_q, 576] into cache positions L_b - s_q + s (programmatic dependent launch).
 cudaError_t launch_append(const void* kv_new, void* kcache, int64_t num_pages, const int32_t* block_table,
                           int64_t bt_stride, const int32_t* seqlens, int batch, int s_q, int* err,
                           cudaStream_t stream);
+// Same positions as launch_append; kv_new (bf16 or fp16) is cast to e5m2 bytes (nearest even, saturating).
+cudaError_t launch_append_fp8(bool bf16, const void* kv_new, void* kcache, int64_t num_pages,
+                              const int32_t* block_table, int64_t bt_stride, const int32_t* seqlens, int batch,
+                              int s_q, int* err, cudaStream_t stream);
 int metadata_smem_bytes(int batch, int num_parts);
 constexpr int kMaxParts = 1024;  // partitions the metadata kernel stages in shared memory
 const void* metadata_kernel_ptr();

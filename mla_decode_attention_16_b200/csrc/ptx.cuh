@@ -9,6 +9,8 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -244,6 +246,17 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem desc] with 8-bit operands (kind::f8f6f4, K = 32 per
+// instruction; A in TMEM holds 4 values per 32-bit column, the lowest K index in the low byte).
+__device__ __forceinline__ void umma_ts_e5m2(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on `bar` when every tcgen05 async op issued so far by this thread completes.
 // Weight-stationary form (M = 32 / 64 / 128): with M = 32 the D tile of N columns is spread over
 // the four TMEM lane quadrants, quadrant q holding rows 0..31 in its lanes and the columns
@@ -330,6 +343,29 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Four 16-bit values (two per word, the lower-indexed in the low half) cast to e5m2, packed
+// four per word with the lowest-indexed value in the low byte (the K order of an A operand in
+// TMEM).  Round to nearest even, saturating to +-57344.
+template <bool kBF16>
+__device__ __forceinline__ uint32_t cast4_e5m2(uint32_t lo_pair, uint32_t hi_pair) {
+  uint32_t a, b;
+  if constexpr (kBF16) {
+    a = __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(lo_pair << 16), __uint_as_float(lo_pair & 0xFFFF0000u)),
+                                 __NV_SATFINITE, __NV_E5M2);
+    b = __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(hi_pair << 16), __uint_as_float(hi_pair & 0xFFFF0000u)),
+                                 __NV_SATFINITE, __NV_E5M2);
+  } else {
+    __half2_raw h0, h1;
+    h0.x = static_cast<unsigned short>(lo_pair & 0xFFFFu);
+    h0.y = static_cast<unsigned short>(lo_pair >> 16);
+    h1.x = static_cast<unsigned short>(hi_pair & 0xFFFFu);
+    h1.y = static_cast<unsigned short>(hi_pair >> 16);
+    a = __nv_cvt_halfraw2_to_fp8x2(h0, __NV_SATFINITE, __NV_E5M2);
+    b = __nv_cvt_halfraw2_to_fp8x2(h1, __NV_SATFINITE, __NV_E5M2);
+  }
+  return (a & 0xFFFFu) | (b << 16);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -379,6 +415,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t smem_addr, uint32_t 
 __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of tcgen05.mma.kind::f8f6f4 with e5m2 A and B (format code 1 in bits
+// 7-9 and 10-12), both K-major, fp32 accumulation; N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_e5m2(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

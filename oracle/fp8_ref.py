@@ -148,14 +148,29 @@ def mla_decode_fp8_ref(
 
     q: [b, s_q, h_q, 576] bf16/fp16 (any dtype exact in fp64); kcache_codes:
     [pages, 64, 1, 576] uint8 e5m2 codes.  The query is cast to e5m2 (the
-    page's q.to(float8_e5m2)), the cache bytes are read as their e5m2 values,
-    and the plain fp64 decode of ``mla_decode_ref`` runs on those values.
+    page's q.to(float8_e5m2)), the bytes of each request's pages are read as
+    their e5m2 values, and the plain fp64 decode of ``mla_decode_ref`` runs on
+    those values, request by request.
     """
     if kcache_codes.dtype != torch.uint8:
         raise ValueError("kcache_codes must hold uint8 e5m2 codes")
+    b, s_q, h_q, _ = q.shape
+    reqs = list(range(b)) if requests is None else [int(r) for r in requests]
     q8 = e5m2_quantize(q.to(_F64))
-    k8 = e5m2_decode(kcache_codes)
-    return mla_decode_ref(q8, k8, block_table, cache_seqlens, softmax_scale, causal, requests=requests)
+    out = torch.zeros(len(reqs), s_q, h_q, 512, dtype=_F64)
+    lse = torch.full((len(reqs), h_q, s_q), -math.inf, dtype=_F64)
+    for i, r in enumerate(reqs):
+        # only this request's pages are read as e5m2 values; they become pages 0 .. n-1 of its own table
+        seqlen = int(cache_seqlens[r])
+        n = -(-seqlen // 64)
+        pages = block_table[r, :n].to(torch.int64)
+        k8 = e5m2_decode(kcache_codes[pages])
+        table = torch.arange(max(n, 1), dtype=torch.int32)[None]
+        o, l = mla_decode_ref(q8[r:r + 1], k8.reshape(n, 64, 1, 576), table, cache_seqlens[r:r + 1],
+                              softmax_scale, causal)
+        out[i] = o[0]
+        lse[i] = l[0]
+    return out, lse
 
 
 def append_kv_fp8_ref(kcache_codes: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,

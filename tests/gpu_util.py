@@ -20,7 +20,7 @@ def run_gpu(inp, num_sm_parts=None, device="cuda"):
     sl = inp.cache_seqlens.to(device)
     b, s_q, h_q, _ = q.shape
     rows = s_q * h_q
-    parts = num_sm_parts or mla.mla_get_num_sm_parts(rows)
+    parts = num_sm_parts or mla.mla_get_num_sm_parts(rows, kv_fp8=inp.kcache.dtype == torch.uint8)
     meta, ns = mla.mla_get_metadata(sl, rows, parts)
     ws = mla.alloc_workspace(b, rows, parts, device)
     out, lse = mla.mla_decode_fwd(q, kc, bt, sl, inp.softmax_scale, inp.causal, meta, ns, ws)

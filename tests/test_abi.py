@@ -85,3 +85,25 @@ def test_host_validation_before_any_launch(L):
     parts = ctypes.c_int()
     assert L.mla_get_num_sm_parts(0, 0, ctypes.byref(parts)) == 1
     assert L.mla_get_num_sm_parts(0, 4096, ctypes.byref(parts)) == 2
+
+
+def test_fp8_cache_flag_validation(L):
+    """MLA_KV_FP8_E5M2 (0x100) is accepted only OR-ed into bf16 / fp16; checks run before any launch."""
+    vp = ctypes.c_void_p
+    fake = vp(256)
+    flag = 0x100
+    # a bad base dtype with the flag, or a stray bit, is rejected as an invalid argument
+    for bad in (flag | 7, 0x200, flag | 0x200):
+        rc = L.mla_decode_fwd(fake, fake, 1, fake, 1, fake, 1, 1, 16, bad, 0.1, 0, fake, fake, 1, fake, 1 << 30,
+                              fake, fake, None)
+        assert rc == 1, hex(bad)
+    # a valid flagged dtype gets as far as the workspace check
+    rc = L.mla_decode_fwd(fake, fake, 1, fake, 1, fake, 4, 1, 16, flag | 1, 0.1, 0, fake, fake, 1, fake, 16,
+                          fake, fake, None)
+    assert rc == 3
+    parts = ctypes.c_int()
+    L.mla_get_num_sm_parts_dtype.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+    assert L.mla_get_num_sm_parts_dtype(0, 16, 7, ctypes.byref(parts)) == 1
+    assert L.mla_get_num_sm_parts_dtype(0, 0, flag, ctypes.byref(parts)) == 1
+    assert L.mla_get_num_sm_parts_dtype(0, 4096, flag, ctypes.byref(parts)) == 2
+    assert L.mla_get_num_sm_parts_dtype(0, 16, flag, None) == 1

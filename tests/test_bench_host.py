@@ -75,7 +75,7 @@ def test_every_bench_workload_has_a_profile_summary():
     for name in WORKLOADS:
         if name == "tiny":
             continue
-        kernel, _ = bench.kernel_of(WORKLOADS[name].rows)
+        kernel, _ = bench.kernel_of(WORKLOADS[name].rows, kv_fp8=WORKLOADS[name].kv_fp8)
         assert os.path.exists(os.path.join(ROOT, "profiles", f"{kernel}_{name}.md")), name
 
 

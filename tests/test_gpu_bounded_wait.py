@@ -37,12 +37,16 @@ def _hook(lib, enable, cycles):
     (3, 1, 16, [700, 64, 2000], False, 1, "few-rows-one-cta"),
     (3, 1, 16, [700, 64, 2000], False, 1, "few-rows-pair"),
     (2, 2, 64, [900, 300], True, 2, "row-tile-pair"),
+    (3, 1, 16, [700, 64, 2000], False, 3, "fp8-cache"),
 ], ids=lambda c: c[-1])
 def test_withheld_arrival_times_out_and_launch_returns(case):
     import mla_decode_attention_16_b200 as mla
 
     b, s_q, h_q, lens, causal, seed, variant = case
-    inp = make_case(b, s_q, h_q, lens, causal=causal, seed=300 + seed)
+    kv_fp8 = variant == "fp8-cache"  # the e5m2-cache kernel (kernel variants do not apply to it)
+    inp = make_case(b, s_q, h_q, lens, causal=causal, seed=300 + seed, kv_fp8=kv_fp8)
+    ref = oracle.mla_decode_fp8_ref if kv_fp8 else oracle.mla_decode_ref
+    variant = "auto" if kv_fp8 else variant
     mla.mla_set_kernel_variant(variant)
     _hook(mla.lib, 1, WAIT_CYCLES)
     try:
@@ -61,8 +65,7 @@ def test_withheld_arrival_times_out_and_launch_returns(case):
     finally:
         mla.mla_set_kernel_variant("auto")
     assert flags[0] == 0, flags
-    ref_out, ref_lse = oracle.mla_decode_ref(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens,
-                                             inp.softmax_scale, inp.causal)
+    ref_out, ref_lse = ref(inp.q, inp.kcache, inp.block_table, inp.cache_seqlens, inp.softmax_scale, inp.causal)
     compare(out, lse, ref_out, ref_lse, f"after timeout {case[:3]}")
 
 

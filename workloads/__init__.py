@@ -19,6 +19,11 @@ varlen-mtp      132    2   128  uniform int in [1,16384] bf16    1.0        yes
 long-fp16        16    2    64  32768 + uniform [-2048,2048] fp16 0.5       yes
 =============== ===== ==== ==== ======================== ======= ========== ======
 
+``memory-bound-fp8`` is ``memory-bound`` with an e5m2 cache (one byte per value).  An e5m2
+cache is drawn as raw codes (no rounding of any number happens here): sign and 2-bit mantissa
+uniform, exponent field uniform in [10, 16] (magnitudes 2^-5 .. 3.5, a spread like the 16-bit
+caches' N(0, 1)); its poison is code 0x71 (10240).
+
 Page pools: ``tiny`` has its 4 pages plus 4 unreferenced pages filled with 1e4;
 ``memory-bound`` uses exactly 4096 pages with ``randperm(4096)`` as its table;
 ``compute-bound`` 8192 pages in random order; the two variable-length workloads
@@ -56,6 +61,7 @@ class Workload:
     pool_kind: str = "exact"  # "exact" | "shared"
     extra_poison_pages: int = 0
     description: str = ""
+    kv_fp8: bool = False  # cache of e5m2 codes (uint8) instead of ``dtype``
 
     @property
     def rows(self) -> int:
@@ -70,6 +76,8 @@ WORKLOADS: Dict[str, Workload] = {
                  description="batch 1, s_q 1, h_q 16, seqlen 256, bf16"),
         Workload("memory-bound", 64, 1, 16, torch.bfloat16, 1.0, False, 1001, "fixed", 4096,
                  description="batch 64, s_q 1, h_q 16, seqlen 4096, bf16"),
+        Workload("memory-bound-fp8", 64, 1, 16, torch.bfloat16, 1.0, False, 1005, "fixed", 4096,
+                 description="batch 64, s_q 1, h_q 16, seqlen 4096, bf16 q, e5m2 cache", kv_fp8=True),
         Workload("compute-bound", 128, 1, 128, torch.bfloat16, 1.0, False, 1002, "fixed", 4096,
                  description="batch 128, s_q 1, h_q 128, seqlen 4096, bf16"),
         Workload("varlen-mtp", 132, 2, 128, torch.bfloat16, 1.0, True, 1003, "uniform", 1, 16384,
@@ -120,6 +128,25 @@ def _randn(g: torch.Generator, shape: Sequence[int], std: float, dtype: torch.dt
     return out
 
 
+E5M2_POISON_CODE = 0x71  # 1.25 * 2^13 = 10240
+
+
+def _rand_e5m2_codes(g: torch.Generator, shape: Sequence[int]) -> torch.Tensor:
+    """uint8 e5m2 codes: random sign and mantissa, exponent field in [10, 16], drawn in slabs."""
+    shape = tuple(int(s) for s in shape)
+    out = torch.empty(shape, dtype=torch.uint8)
+    flat = out.view(shape[0], -1)
+    step = max(1, (1 << 24) // max(1, flat.shape[1]))
+    for i in range(0, shape[0], step):
+        j = min(shape[0], i + step)
+        n = (j - i, flat.shape[1])
+        sign = torch.randint(0, 2, n, generator=g, dtype=torch.int32)
+        expo = torch.randint(10, 17, n, generator=g, dtype=torch.int32)
+        mant = torch.randint(0, 4, n, generator=g, dtype=torch.int32)
+        flat[i:j] = ((sign << 7) | (expo << 2) | mant).to(torch.uint8)
+    return out
+
+
 def make_case(
     batch: int,
     s_q: int,
@@ -134,12 +161,14 @@ def make_case(
     table_pad: int = 0,
     poison_tail: bool = True,
     softmax_scale: Optional[float] = None,
+    kv_fp8: bool = False,
 ) -> Inputs:
     """Build one seeded paged-cache case with the given per-request lengths.
 
     Pages are drawn for every request (ceil(L/64) each), the pool is shuffled
     with ``randperm`` and ``extra_poison_pages`` unreferenced pages filled with
     1e4 are mixed in.  ``table_pad`` extra -1 columns are appended to the table.
+    ``kv_fp8``: the cache is uint8 e5m2 codes (poison code 0x71 = 10240).
     """
     g = torch.Generator().manual_seed(int(seed))
     seqlens = [int(x) for x in seqlens]
@@ -149,7 +178,12 @@ def make_case(
     pool = used + int(extra_poison_pages)
     width = max([1] + n_pages) + int(table_pad)
     q = _randn(g, (batch, s_q, h_q, D_K), std, dtype)
-    kcache = _randn(g, (max(pool, 1), PAGE, 1, D_K), std, dtype)
+    if kv_fp8:
+        kcache = _rand_e5m2_codes(g, (max(pool, 1), PAGE, 1, D_K))
+        poison = torch.tensor(E5M2_POISON_CODE, dtype=torch.uint8)
+    else:
+        kcache = _randn(g, (max(pool, 1), PAGE, 1, D_K), std, dtype)
+        poison = torch.tensor(POISON, dtype=dtype)
     perm = torch.randperm(max(pool, 1), generator=g)
     table = torch.full((batch, width), -1, dtype=torch.int32)
     pos = 0
@@ -158,12 +192,12 @@ def make_case(
         pos += n
     # unreferenced pages of the pool are poison
     if pool > used:
-        kcache[perm[used:pool]] = torch.tensor(POISON, dtype=dtype)
+        kcache[perm[used:pool]] = poison
     # slots past L in a request's last page are poison too
     if poison_tail:
         for r, L in enumerate(seqlens):
             if L % PAGE:
-                kcache[int(table[r, n_pages[r] - 1]), L % PAGE:] = torch.tensor(POISON, dtype=dtype)
+                kcache[int(table[r, n_pages[r] - 1]), L % PAGE:] = poison
     scale = D_K ** -0.5 if softmax_scale is None else float(softmax_scale)
     return Inputs(q, kcache, table, torch.tensor(seqlens, dtype=torch.int32), scale, causal,
                   meta={"seed": seed, "pool_pages": pool, "used_pages": used})
@@ -185,28 +219,34 @@ def make_workload(name: str) -> Inputs:
     w = WORKLOADS[name]
     g = torch.Generator().manual_seed(w.seed)
     seqlens = draw_seqlens(w, g)
-    if name == "memory-bound":
+    if name in ("memory-bound", "memory-bound-fp8"):
         # exactly the 4096-page pool, table = randperm(4096) viewed as [64, 64]
         q = _randn(g, (w.batch, w.s_q, w.h_q, D_K), w.std, w.dtype)
-        kcache = _randn(g, (4096, PAGE, 1, D_K), w.std, w.dtype)
+        if w.kv_fp8:
+            kcache = _rand_e5m2_codes(g, (4096, PAGE, 1, D_K))
+        else:
+            kcache = _randn(g, (4096, PAGE, 1, D_K), w.std, w.dtype)
         table = torch.randperm(4096, generator=g).to(torch.int32).view(64, 64).contiguous()
         return Inputs(q, kcache, table, torch.tensor(seqlens, dtype=torch.int32), D_K ** -0.5, w.causal,
                       meta={"seed": w.seed, "pool_pages": 4096, "used_pages": 4096})
     return make_case(w.batch, w.s_q, w.h_q, seqlens, dtype=w.dtype, std=w.std, causal=w.causal,
-                     seed=w.seed + 7919, extra_poison_pages=w.extra_poison_pages)
+                     seed=w.seed + 7919, extra_poison_pages=w.extra_poison_pages, kv_fp8=w.kv_fp8)
 
 
-def algorithmic_cost(seqlens: Sequence[int], s_q: int, h_q: int, elem_bytes: int = 2) -> Dict[str, float]:
+def algorithmic_cost(seqlens: Sequence[int], s_q: int, h_q: int, elem_bytes: int = 2,
+                     kv_elem_bytes: Optional[int] = None) -> Dict[str, float]:
     """FLOPs and bytes of one decode call by the pages' cost model.
 
-    FLOPs = 2 * h_q * s_q * (576 + 512) * sum(L); bytes = 576 * elem * sum(L)
-    (each cached row read once, V being part of it) + q + out + lse.
+    FLOPs = 2 * h_q * s_q * (576 + 512) * sum(L); bytes = 576 * kv_elem * sum(L)
+    (each cached row read once, V being part of it) + q + out + lse (elem bytes each;
+    kv_elem defaults to elem, 1 for an e5m2 cache).
     """
+    kv_elem = elem_bytes if kv_elem_bytes is None else kv_elem_bytes
     tot = float(sum(int(x) for x in seqlens))
     b = len(seqlens)
     rows = s_q * h_q
     flops = 2.0 * rows * (576 + 512) * tot
-    kv_bytes = 576.0 * elem_bytes * tot
+    kv_bytes = 576.0 * kv_elem * tot
     io_bytes = b * rows * (576 * elem_bytes + 512 * elem_bytes + 4)
     return {"flops": flops, "kv_bytes": kv_bytes, "bytes": kv_bytes + io_bytes, "tokens": tot}
 
@@ -218,4 +258,4 @@ def seqlens_of(name: str) -> List[int]:
 
 
 __all__ = ["WORKLOADS", "Workload", "Inputs", "make_case", "make_workload", "algorithmic_cost",
-           "seqlens_of", "POISON", "PAGE", "D_K"]
+           "seqlens_of", "POISON", "E5M2_POISON_CODE", "PAGE", "D_K"]
