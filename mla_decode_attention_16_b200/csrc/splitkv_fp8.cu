@@ -33,11 +33,16 @@
 // them through L2.
 //
 // Roles (384 threads): warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0
-// issues every tcgen05.mma; warps 2-3 widen V; warps 4-7: warp 4 + (chunk & 1)
+// issues the Q.K^T MMAs; warps 2-3 widen V; warps 4-7: warp 4 + (chunk & 1)
 // runs a chunk's softmax (one thread per query row), all four rescale O when a
-// row's exponent reference moves; warps 8-11 write each chunk's epilogue, and
-// warps 8 / 9 cast and load Q for even / odd chunks (Q of consecutive chunks in
-// lane quadrants 0 / 1, so the next chunk's Q is written while one runs).
+// row's exponent reference moves, and warp 6 lane 0 issues the P.V MMAs; warps
+// 8-11 write each chunk's epilogue, and warps 8 / 9 cast and load Q for even /
+// odd chunks (Q of consecutive chunks in lane quadrants 0 / 1, so the next
+// chunk's Q is written while one runs).  Two issuing threads: one thread
+// issuing every MMA (~65 cycles per Q.K^T and ~100 per weight-stationary P.V
+// instruction, plus its waits and commits) was the bottleneck at ~3,400 cycles
+// per page while the tensor pipe was busy for ~900; tcgen05.commit tracks the
+// issuing thread's own MMAs, so each issuer commits its own barriers.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -61,7 +66,6 @@ constexpr int kStageBytes = 4 * kBox8 + kBoxR;  // 36 KB: one page
 constexpr int kStages = 4;
 constexpr int kVBox = kPage * 128;              // 8 KB: one page x 64 fp16 values
 constexpr int kQCols = kDK / 4;                 // 144 TMEM columns: 4 e5m2 values each
-constexpr int kConvThreads = 64;                // warps 2-3
 constexpr float kRescaleThreshold = 8.0f;       // see splitkv.cu
 
 enum Bar {
@@ -79,7 +83,8 @@ enum Bar {
   kOFinal,                       // one phase per chunk
   kOEmpty,                       // count 4: epilogue finished reading O
   kStats = kOEmpty + 1,          // [2] row sums / reference maxima of a chunk parity in smem
-  kDrain = kStats + 2,
+  kDrain = kStats + 2,           // Q.K^T issuer's tensor-core work drained
+  kDrainPV,                      // P.V issuer's tensor-core work drained
   kNumBars
 };
 
@@ -198,6 +203,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int br = meta[0], bk = meta[1], er = meta[2], ek = meta[3], bs = meta[4];
   int* err = p.err;
 
+  // O[:, 256h ..] += P[:, 16kk ..] . V16[16kk .., 256h ..] for page itp (chunk-relative index jjp of
+  // chunk `chunk`), issued by warp 6 lane 0 once the four softmax warps have released P.
+  // A = P (32 rows, K-major), B = V16 (MN-major view of value boxes 4h .. 4h+3, 8 KB apart; 16
+  // keys = 2 x 1 KB).
+  auto issue_pv = [&](uint32_t itp, int jjp, bool last, uint32_t chunk) {
+    constexpr uint32_t idesc_pv = idesc_f16(false, 32, 256, false, true);  // fp16 P and V
+    const uint32_t vbase = sbase + Lay::kOffV;
+    const int b = itp & 1;
+    if (jjp == 0) mbar_wait(bar(kOEmpty), (chunk & 1) ^ 1, wctl, err, kDevErrTimeout);
+    mbar_wait(bar(kPFull + b), (itp >> 1) & 1, wctl, err, kDevErrTimeout);
+    const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      mbar_wait(bar(kVFull + h), itp & 1, wctl, err, kDevErrTimeout);
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kPage / 16; ++kk) {
+        const uint64_t adesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
+        const uint64_t bdesc = smem_desc_sw128(vbase + (4 * h) * kVBox + kk * 2048, kVBox, 1024);
+        umma_ws_ss(tmem + Lay::kColO + 64 * h, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(bar(kVEmpty + h));
+    }
+    umma_commit(bar(kPEmpty + b));
+    umma_commit(bar(kODone));
+    if (last) umma_commit(bar(kOFinal));
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (pages only)
     if (lane == 0) {
@@ -233,35 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(bar(kKvFull + j % kStages), (j / kStages) & 1, wctl->limit);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Q.K^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_e5m2(128, kPage);
-      constexpr uint32_t idesc_pv = idesc_f16(false, 32, 256, false, true);  // fp16 P and V
-      const uint32_t vbase = sbase + Lay::kOffV;
       uint32_t it = 0, chunk = 0;
-      auto issue_pv = [&](uint32_t itp, int jjp, bool last) {
-        const int b = itp & 1;
-        if (jjp == 0) mbar_wait(bar(kOEmpty), (chunk & 1) ^ 1, wctl, err, kDevErrTimeout);
-        mbar_wait(bar(kPFull + b), (itp >> 1) & 1, wctl, err, kDevErrTimeout);
-        const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          mbar_wait(bar(kVFull + h), itp & 1, wctl, err, kDevErrTimeout);
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kPage / 16; ++kk) {
-            // O[:, 256h ..] += P[:, 16kk ..] . V16[16kk .., 256h ..]: A = P (32 rows, K-major), B = V16
-            // (MN-major view of value boxes 4h .. 4h+3, 8 KB apart; 16 keys = 2 x 1 KB)
-            const uint64_t adesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(vbase + (4 * h) * kVBox + kk * 2048, kVBox, 1024);
-            umma_ws_ss(tmem + Lay::kColO + 64 * h, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(bar(kVEmpty + h));
-        }
-        umma_commit(bar(kPEmpty + b));
-        umma_commit(bar(kODone));
-        if (last) umma_commit(bar(kOFinal));
-      };
       int cur = br;
       Chunk ch;
       while (!aborted(wctl) && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
@@ -276,7 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, wctl, err, kDevErrTimeout);
           tc_fence_after();
           const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
-#pragma unroll 1
+          // fully unrolled: the descriptors become constants plus the stage base (a rolled loop
+          // that picks the box form at run time spent ~95 extra cycles per MMA in this thread,
+          // the kernel's bottleneck)
+#pragma unroll
           for (int s = 0; s < kDK / 32; ++s) {
             // 32 columns per MMA: columns 0..511 from the four 128-column boxes (4 steps of 32
             // bytes each), 512..575 from the 64-column box (2 steps)
@@ -287,9 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(bar(kSFull));
           umma_commit(bar(kKvEmpty + st));
           if (jj == nb - 1) umma_commit(bar(kQEmpty + qpar));
-          if (jj > 0) issue_pv(itc - 1, jj - 1, false);
         }
-        issue_pv(it + nb - 1, nb - 1, true);
         it += nb;
         ++chunk;
       }
@@ -312,27 +321,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           mbar_wait(bar(kVEmpty + h), (it & 1) ^ 1, wctl, err, kDevErrTimeout);
-          // values 256h .. 256h+255 = e5m2 boxes 2h, 2h+1 (64 rows x 8 16-byte pieces each), each
-          // piece written as two fp16 pieces.  16-byte accesses are served 8 threads at a time: those
-          // 8 threads take 8 consecutive rows of one logical piece c, so with the 128-byte swizzle
-          // (physical piece = logical ^ (row & 7)) their loads and each of their two stores fall
-          // on 8 different 16-byte bank groups
-#pragma unroll 4
+          // values 256h .. 256h+255 = e5m2 boxes 2h, 2h+1: thread ct widens key row ct of both boxes
+          // (8 16-byte pieces each; piece c holds values 128i + 16c .., stored at piece c ^ (row & 7)
+          // by the 128-byte swizzle) into fp16 boxes 4h .. 4h+3 (each e5m2 byte b is the fp16 with
+          // bits b << 8).  All 16 loads are issued before the first store, so they overlap instead
+          // of each waiting behind the stores before it.  16-byte accesses are served 8 threads
+          // at a time, here 8 consecutive rows: the XOR swizzle spreads their loads and each of
+          // their two stores over 8 different 16-byte bank groups.
+          const int k = ct;
+          uint4 xs[16];
+#pragma unroll
           for (int n = 0; n < 16; ++n) {
-            const int u = ct + kConvThreads * n;        // 0 .. 1023
-            const int i = 2 * h + (u >> 9);             // e5m2 box
-            const int k = (u & 0x38) + (u & 7);         // key (row of the box): 8 row groups x 8 rows
-            const int c = (u >> 6) & 7;                 // logical piece: values 128i + 16c ..
-            const int pc = c ^ (k & 7);                 // physical 16-byte piece in the row
-            const uint4 x = *reinterpret_cast<const uint4*>(kst + i * kBox8 + k * 128 + pc * 16);
-            // e5m2 byte b is the fp16 with bits b << 8
+            const int i = 2 * h + (n >> 3), c = n & 7;
+            xs[n] = *reinterpret_cast<const uint4*>(kst + i * kBox8 + k * 128 + ((c ^ (k & 7)) << 4));
+          }
+#pragma unroll
+          for (int n = 0; n < 16; ++n) {
+            const int i = 2 * h + (n >> 3), c = n & 7;
+            const uint4 x = xs[n];
             const uint4 lo = make_uint4(__byte_perm(x.x, 0, 0x1404), __byte_perm(x.x, 0, 0x3424),
                                         __byte_perm(x.y, 0, 0x1404), __byte_perm(x.y, 0, 0x3424));
             const uint4 hi = make_uint4(__byte_perm(x.z, 0, 0x1404), __byte_perm(x.z, 0, 0x3424),
                                         __byte_perm(x.w, 0, 0x1404), __byte_perm(x.w, 0, 0x3424));
-            const int vb = 2 * i + (c >> 2);            // fp16 box of values 64 vb .. 64 vb + 63
-            const int j0 = 2 * (c & 3);                 // logical fp16 pieces j0, j0 + 1 of the row
-            uint8_t* row = vdst + vb * kVBox + k * 128;
+            const int j0 = 2 * (c & 3);  // logical fp16 pieces j0, j0 + 1 of the row in box 2i + c / 4
+            uint8_t* row = vdst + (2 * i + (c >> 2)) * kVBox + k * 128;
             *reinterpret_cast<uint4*>(row + ((j0 ^ (k & 7)) << 4)) = lo;
             *reinterpret_cast<uint4*>(row + (((j0 + 1) ^ (k & 7)) << 4)) = hi;
           }
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax (one warp per chunk) + O rescale
+    // ------------------------------------------------------------ softmax (one warp per chunk) + O rescale + P.V issue
     const int q4 = warp & 3;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int r = lane;
@@ -449,6 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kPFull + b));
+        if (warp == 6) {  // this page's P.V (after all four warps arrived: P written, O rescaled)
+          if (lane == 0 && !aborted(wctl)) issue_pv(itc, jj, jj == nb - 1, chunk);
+          __syncwarp();
+        }
       }
       if (smx) {
         if (r < NP) {
@@ -460,6 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       it += nb;
       ++chunk;
+    }
+    if (warp == 6 && lane == 0) {
+      umma_commit(bar(kDrainPV));
+      mbar_wait_drain(bar(kDrainPV), 0, wctl->limit);
     }
   } else {
     // ------------------------------------------------------------ Q loads (warps 8 / 9) and epilogue (8-11)

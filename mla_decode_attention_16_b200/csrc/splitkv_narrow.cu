@@ -27,10 +27,14 @@
 // ignored).
 //
 // Roles (384 threads): warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0
-// issues every tcgen05.mma; warps 4-7: warp 4 + (chunk & 1) runs the softmax
-// of a chunk (one thread per query row) and all four rescale O when a row's
-// exponent reference moves; warps 8-11 write each chunk's epilogue, and warps
-// 8 / 9 load Q for even / odd chunks.
+// issues the Q.K^T MMAs; warps 4-7: warp 4 + (chunk & 1) runs the softmax of a
+// chunk (one thread per query row), all four rescale O when a row's exponent
+// reference moves, and warp 6 lane 0 issues the P.V MMAs; warps 8-11 write each
+// chunk's epilogue, and warps 8 / 9 load Q for even / odd chunks.  With one
+// thread issuing both products, a page's P.V had to wait behind the next page's
+// Q.K^T, holding the page's 72 KB stage that much longer; with two issuers P.V
+// goes as soon as P is written (tcgen05.commit tracks the issuing thread's own
+// MMAs, so each issuer commits its own barriers).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -66,7 +70,8 @@ enum Bar {
   kOFinal,                      // [2] one phase per chunk using that O buffer
   kOEmpty = kOFinal + 2,        // [2] epilogue finished reading that O buffer
   kStats = kOEmpty + 2,         // [2] row sums / reference maxima of a chunk parity in smem
-  kDrain = kStats + 2,
+  kDrain = kStats + 2,          // Q.K^T issuer's tensor-core work drained
+  kDrainPV,                     // P.V issuer's tensor-core work drained
   kNumBars
 };
 
@@ -171,6 +176,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int R = p.rows;
   int* err = p.err;
 
+  // O[:, 256h ..] += P[:, 16kk ..] . V[16kk .., 256h ..] for page itp (chunk-relative index jjp of
+  // chunk `chunk`), issued by warp 6 lane 0 once the four softmax warps have released P.  A = P (32
+  // rows, K-major), B = V (MN-major view of the page's column boxes 4h .. 4h+3, 8 KB apart; 16 keys
+  // = 2 x 1 KB).  Its commit also frees the page stage: the page's Q.K^T, issued by the other
+  // thread, completed before its softmax could write P.
+  auto issue_pv = [&](uint32_t itp, int jjp, bool last, uint32_t chunk) {
+    constexpr uint32_t idesc_pv = idesc_f16(kBF16, 32, 256, false, true);
+    const int st = itp % kStages;
+    const int b = itp & 1;
+    const int ob = chunk % kOBufs;
+    if (jjp == 0) mbar_wait(bar(kOEmpty + ob), ((chunk / kOBufs) & 1) ^ 1, wctl, err, kDevErrTimeout);
+    mbar_wait(bar(kPFull + b), (itp >> 1) & 1, wctl, err, kDevErrTimeout);
+    tc_fence_after();
+    const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
+    const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
+    const uint32_t dcol = tmem + Lay::kColO + ob * 128;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int kk = 0; kk < kPage / 16; ++kk) {
+        const uint64_t adesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
+        const uint64_t bdesc = smem_desc_sw128(kst + (4 * h) * kKBox + kk * 2048, kKBox, 1024);
+        umma_ws_ss(dcol + 64 * h, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
+      }
+    }
+    umma_commit(bar(kKvEmpty + st));
+    umma_commit(bar(kPEmpty + b));
+    umma_commit(bar(kODone));
+    if (last) umma_commit(bar(kOFinal + ob));
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (pages only)
     if (lane == 0) {
@@ -205,37 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(bar(kKvFull + j % kStages), (j / kStages) & 1, wctl->limit);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Q.K^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16(kBF16, 128, kPage, false, false);
-      constexpr uint32_t idesc_pv = idesc_f16(kBF16, 32, 256, false, true);
       uint32_t it = 0, chunk = 0;
-      auto issue_pv = [&](uint32_t itp, int jjp, bool last) {
-        const int st = itp % kStages;
-        const int b = itp & 1;
-        const int ob = chunk % kOBufs;
-        if (jjp == 0) mbar_wait(bar(kOEmpty + ob), ((chunk / kOBufs) & 1) ^ 1, wctl, err, kDevErrTimeout);
-        mbar_wait(bar(kPFull + b), (itp >> 1) & 1, wctl, err, kDevErrTimeout);
-        tc_fence_after();
-        const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
-        const uint32_t pbuf = sbase + Lay::kOffP + b * Lay::kPBytes;
-        const uint32_t dcol = tmem + Lay::kColO + ob * 128;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < kPage / 16; ++kk) {
-            // O[:, 256h ..] += P[:, 16kk ..] . V[16kk .., 256h ..]: A = P (32 rows, K-major), B = V
-            // (MN-major view of column boxes 4h .. 4h+3, 8 KB apart; 16 keys = 2 x 1 KB)
-            const uint64_t adesc = smem_desc_sw128(pbuf + kk * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(kst + (4 * h) * kKBox + kk * 2048, kKBox, 1024);
-            umma_ws_ss(dcol + 64 * h, adesc, bdesc, idesc_pv, (jjp > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        umma_commit(bar(kKvEmpty + st));
-        umma_commit(bar(kPEmpty + b));
-        umma_commit(bar(kODone));
-        if (last) umma_commit(bar(kOFinal + ob));
-      };
       int cur = br;
       Chunk ch;
       while (!aborted(wctl) && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
@@ -250,8 +259,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, wctl, err, kDevErrTimeout);
           tc_fence_after();
           const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
-#pragma unroll 1
+          // fully unrolled: the descriptors become constants plus the stage base, which keeps this
+          // single issuing thread -- the kernel's bottleneck -- at ~1 MMA per tcgen05.mma slot
+#pragma unroll
           for (int i = 0; i < kBoxes; ++i) {
+#pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const int s = 4 * i + kk;
               const uint64_t bdesc = smem_desc_sw128(kst + i * kKBox + kk * 32, 16, 1024);
@@ -260,9 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           umma_commit(bar(kSFull));
           if (jj == nb - 1) umma_commit(bar(kQEmpty + qpar));
-          if (jj > 0) issue_pv(itc - 1, jj - 1, false);
         }
-        issue_pv(it + nb - 1, nb - 1, true);
         it += nb;
         ++chunk;
       }
@@ -270,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(bar(kDrain), 0, wctl->limit);
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ softmax (one warp per chunk) + O rescale
+    // ------------------------------------------------------------ softmax (one warp per chunk) + O rescale + P.V issue
     const int q4 = warp & 3;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int r = lane;
@@ -375,6 +385,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kPFull + b));
+        if (warp == 6) {  // this page's P.V (after all four warps arrived: P written, O rescaled)
+          if (lane == 0 && !aborted(wctl)) issue_pv(itc, jj, jj == nb - 1, chunk);
+          __syncwarp();
+        }
       }
       if (smx) {
         // this stats slot was last used by chunk - 2; with two O buffers its epilogue may still
@@ -390,6 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       it += nb;
       ++chunk;
+    }
+    if (warp == 6 && lane == 0) {
+      umma_commit(bar(kDrainPV));
+      mbar_wait_drain(bar(kDrainPV), 0, wctl->limit);
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ Q loads (warps 8 / 9) and epilogue (8-11)
