@@ -21,6 +21,8 @@
 //                      the page stage into a 64 KB shared-memory tile laid out as
 //                      the 16-bit kernels' page boxes (128-byte swizzle)
 //   O [rows x 512]  += P16 . V16  weight-stationary M = 32, N = 256: 8 MMAs
+// S is double-buffered in TMEM (the query in e5m2 takes only 144 columns), so the
+// next page's Q.K^T is issued while the softmax still works on this one.
 // The page stage is released once its Q.K^T and its conversion are done (not
 // after the P.V that follows the next page), so four 36 KB stages keep about
 // three pages in flight per SM.  V16 is converted in two halves of 256 values,
@@ -73,9 +75,9 @@ enum Bar {
   kKvEmpty = kKvFull + kStages,  // count 3: the Q.K^T commit + one arrival per converter warp
   kQFull = kKvEmpty + kStages,   // [2] Q rows of a chunk parity written to TMEM
   kQEmpty = kQFull + 2,          // [2] last Q.K^T of a chunk of that parity completed
-  kSFull = kQEmpty + 2,
-  kSEmpty,
-  kPFull,                        // [2] count 4
+  kSFull = kQEmpty + 2,          // [2] S buffer of page parity b written
+  kSEmpty = kSFull + 2,          // [2] S buffer read by the softmax
+  kPFull = kSEmpty + 2,                        // [2] count 4
   kPEmpty = kPFull + 2,          // [2]
   kVFull = kPEmpty + 2,          // [2] half h of V16 written (count 2: one per converter warp)
   kVEmpty = kVFull + 2,          // [2] the P.V MMAs that read half h completed
@@ -104,8 +106,8 @@ struct Layout {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 0;  // O: 2 halves of 256 values x 64 columns (see umma_ws_ss)
-  static constexpr uint32_t kColS = kColO + 128;
-  static constexpr uint32_t kColQ = kColS + kPage;
+  static constexpr uint32_t kColS = kColO + 128;  // S: two buffers of 64 columns (page parity)
+  static constexpr uint32_t kColQ = kColS + 2 * kPage;
   static_assert(kColQ + kQCols <= kTmemCols, "TMEM budget");
 };
 
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t itc = it + jj;
           const int st = itc % kStages;
           mbar_wait(bar(kKvFull + st), (itc / kStages) & 1, wctl, err, kDevErrTimeout);
-          mbar_wait(bar(kSEmpty), (itc & 1) ^ 1, wctl, err, kDevErrTimeout);
+          mbar_wait(bar(kSEmpty + (itc & 1)), ((itc >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
           tc_fence_after();
           const uint32_t kst = sbase + Lay::kOffK + st * kStageBytes;
           // fully unrolled: the descriptors become constants plus the stage base (a rolled loop
@@ -293,9 +295,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // bytes each), 512..575 from the 64-column box (2 steps)
             const uint64_t bdesc = s < 16 ? smem_desc_sw128(kst + (s >> 2) * kBox8 + (s & 3) * 32, 16, 1024)
                                           : smem_desc_sw64(kst + 4 * kBox8 + (s - 16) * 32, 16, 512);
-            umma_ts_e5m2(tmem + Lay::kColS, tmem + Lay::kColQ + 8 * s, bdesc, idesc_qk, s > 0 ? 1u : 0u);
+            umma_ts_e5m2(tmem + Lay::kColS + kPage * (itc & 1), tmem + Lay::kColQ + 8 * s, bdesc, idesc_qk,
+                         s > 0 ? 1u : 0u);
           }
-          umma_commit(bar(kSFull));
+          umma_commit(bar(kSFull + (itc & 1)));
           umma_commit(bar(kKvEmpty + st));
           if (jj == nb - 1) umma_commit(bar(kQEmpty + qpar));
         }
@@ -361,6 +364,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int r = lane;
+    // With 16 query rows, lanes r and r + 16 share row r: the Q loader writes every row into both
+    // halves of its lane quadrant, so S holds each row twice and each lane takes 32 of its 64 keys
+    // (half the work and registers of one lane per row); the row's maximum and sum combine over
+    // the pair with one shuffle each.
+    constexpr int kSplit = NP == 16 ? 2 : 1;
+    constexpr int kKeys = kPage / kSplit;  // keys per lane
+    const int row = kSplit == 2 ? (lane & 15) : lane;
+    const int half = kSplit == 2 ? (lane >> 4) : 0;
     uint32_t it = 0, chunk = 0;
     int cur = br;
     Chunk ch;
@@ -369,8 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int par = chunk & 1;
       const bool smx = q4 == par;  // warp 4 for even chunks, warp 5 for odd ones (lane quadrant = parity)
       int limit = 0;
-      if (smx && r < Rt) {
-        limit = p.causal ? ch.L - (p.s_q - 1 - (r0 + r) / p.h_q) : ch.L;
+      if (smx && row < Rt) {
+        limit = p.causal ? ch.L - (p.s_q - 1 - (r0 + row) / p.h_q) : ch.L;
         limit = limit < 0 ? 0 : limit;
       }
       float m = -INFINITY, l = 0.f;
@@ -378,33 +389,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t itc = it + jj;
         const int b = itc & 1;
         if (smx) {
-          mbar_wait(bar(kSFull), itc & 1, wctl, err, kDevErrTimeout);
+          mbar_wait(bar(kSFull + b), (itc >> 1) & 1, wctl, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
-          float x[64];
+          float x[kKeys];
           {
+            // tcgen05.ld takes one column address for the whole warp: every lane loads both
+            // 32-column halves and keeps its own (all 64 columns when a lane owns a whole row)
             uint32_t v0[32], v1[32];
-            tmem_ld32(t_lane + Lay::kColS, v0);
-            tmem_ld32(t_lane + Lay::kColS + 32, v1);
+            tmem_ld32(t_lane + Lay::kColS + kPage * b, v0);
+            tmem_ld32(t_lane + Lay::kColS + kPage * b + 32, v1);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              x[c] = __uint_as_float(v0[c]);
-              x[32 + c] = __uint_as_float(v1[c]);
+              if constexpr (kKeys == 64) {
+                x[c] = __uint_as_float(v0[c]);
+                x[32 + c] = __uint_as_float(v1[c]);
+              } else {
+                x[c] = __uint_as_float(half ? v1[c] : v0[c]);
+              }
             }
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kSEmpty));
+          if (lane == 0) mbar_arrive(bar(kSEmpty + b));
 
-          const int kbase = (ch.lo + jj) * kPage;
+          const int kbase = (ch.lo + jj) * kPage + kKeys * half;
           float mx = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
+          for (int c = 0; c < kKeys; ++c) {
             const float t = (kbase + c < limit) ? x[c] * p.scale_log2 : -INFINITY;
             x[c] = t;
             mx = fmaxf(mx, t);
           }
+          if constexpr (kSplit == 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           bool resc = false;
           float alpha = 1.f;
           if (mx > m + kRescaleThreshold) {
@@ -416,25 +434,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float base = (m == -INFINITY) ? 0.f : m;
           float sum = 0.f;
-          uint32_t pk[32];
+          uint32_t pk[kKeys / 2];
 #pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
+          for (int c2 = 0; c2 < kKeys / 2; ++c2) {
             const float p0 = ex2(x[2 * c2] - base);
             const float p1 = ex2(x[2 * c2 + 1] - base);
             sum += p0 + p1;
             pk[c2] = pack_half2(p0, p1);
           }
-          l = l * alpha + sum;
+          l = l * alpha + sum;  // this lane's keys of the row
           const bool any_resc = __any_sync(0xffffffffu, resc);
-          if (r < NP) s_alpha[b * NP + r] = alpha;
+          if (half == 0 && row < NP) s_alpha[b * NP + row] = alpha;
           if (lane == 0) s_flag[b] = any_resc ? 1 : 0;
           mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
-          if (r < NP) {
-            // P row r: 64 keys = 128 bytes, 16-byte pieces XOR-swizzled by row (128-byte swizzle)
-            uint8_t* prow = smem + Lay::kOffP + b * Lay::kPBytes + r * 128;
+          if (row < NP) {
+            // P row: 64 keys = 128 bytes, 16-byte pieces XOR-swizzled by row (128-byte swizzle);
+            // this lane's keys are pieces (kKeys / 8) * half ..
+            uint8_t* prow = smem + Lay::kOffP + b * Lay::kPBytes + row * 128;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<uint4*>(prow + ((k ^ (r & 7)) << 4)) =
+            for (int k = 0; k < kKeys / 8; ++k)
+              *reinterpret_cast<uint4*>(prow + ((((kKeys / 8) * half + k) ^ (row & 7)) << 4)) =
                   make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
           }
           fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
@@ -467,9 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (smx) {
-        if (r < NP) {
-          s_lsum[par * NP + r] = l;
-          s_mref[par * NP + r] = m;
+        float lrow = l;
+        if constexpr (kSplit == 2) lrow += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (half == 0 && row < NP) {
+          s_lsum[par * NP + row] = lrow;
+          s_mref[par * NP + row] = m;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kStats + par));
@@ -491,15 +512,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar(kQEmpty + (idx & 1)), ((idx >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
+      // with 16 rows, lanes r and r + 16 both hold row r (see the softmax)
+      const int qr = NP == 16 ? (r & 15) : r;
       const uint4* qrow = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint16_t*>(qptr) + (static_cast<int64_t>(c.req) * R + r0 + (r < Rt ? r : 0)) * kDK);
+          reinterpret_cast<const uint16_t*>(qptr) + (static_cast<int64_t>(c.req) * R + r0 + (qr < Rt ? qr : 0)) * kDK);
 #pragma unroll 1
       for (int c16 = 0; c16 < kQCols / 16; ++c16) {
         uint32_t w[16];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           uint4 d = make_uint4(0, 0, 0, 0);
-          if (r < Rt) d = __ldg(qrow + c16 * 8 + v);
+          if (qr < Rt) d = __ldg(qrow + c16 * 8 + v);
           w[2 * v] = cast4_e5m2<kBF16>(d.x, d.y);
           w[2 * v + 1] = cast4_e5m2<kBF16>(d.z, d.w);
         }

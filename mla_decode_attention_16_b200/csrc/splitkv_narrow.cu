@@ -284,6 +284,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int r = lane;
+    // With 16 query rows, lanes r and r + 16 share row r: the Q loader writes every row into both
+    // halves of its lane quadrant, so S holds each row twice and each lane takes 32 of its 64 keys
+    // (half the work and registers of one lane per row); the row's maximum and sum combine over
+    // the pair with one shuffle each.
+    constexpr int kSplit = NP == 16 ? 2 : 1;
+    constexpr int kKeys = kPage / kSplit;  // keys per lane
+    const int row = kSplit == 2 ? (lane & 15) : lane;
+    const int half = kSplit == 2 ? (lane >> 4) : 0;
     uint32_t it = 0, chunk = 0;
     int cur = br;
     Chunk ch;
@@ -293,8 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool smx = q4 == par;  // warp 4 for even chunks, warp 5 for odd ones (lane quadrant = parity)
       const int ob = chunk % kOBufs;
       int limit = 0;
-      if (smx && r < R) {
-        limit = p.causal ? ch.L - (p.s_q - 1 - r / p.h_q) : ch.L;
+      if (smx && row < R) {
+        limit = p.causal ? ch.L - (p.s_q - 1 - row / p.h_q) : ch.L;
         limit = limit < 0 ? 0 : limit;
       }
       float m = -INFINITY, l = 0.f;
@@ -305,30 +313,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(kSFull), itc & 1, wctl, err, kDevErrTimeout);
           __syncwarp();
           tc_fence_after();
-          float x[64];
+          float x[kKeys];
           {
-            uint32_t r0[32], r1[32];
-            tmem_ld32(t_lane + Lay::kColS, r0);
-            tmem_ld32(t_lane + Lay::kColS + 32, r1);
+            // tcgen05.ld takes one column address for the whole warp: every lane loads both
+            // 32-column halves and keeps its own (all 64 columns when a lane owns a whole row)
+            uint32_t v0[32], v1[32];
+            tmem_ld32(t_lane + Lay::kColS, v0);
+            tmem_ld32(t_lane + Lay::kColS + 32, v1);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              x[c] = __uint_as_float(r0[c]);
-              x[32 + c] = __uint_as_float(r1[c]);
+              if constexpr (kKeys == 64) {
+                x[c] = __uint_as_float(v0[c]);
+                x[32 + c] = __uint_as_float(v1[c]);
+              } else {
+                x[c] = __uint_as_float(half ? v1[c] : v0[c]);
+              }
             }
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(kSEmpty));
 
-          const int kbase = (ch.lo + jj) * kPage;
+          const int kbase = (ch.lo + jj) * kPage + kKeys * half;
           float mx = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
+          for (int c = 0; c < kKeys; ++c) {
             const float t = (kbase + c < limit) ? x[c] * p.scale_log2 : -INFINITY;
             x[c] = t;
             mx = fmaxf(mx, t);
           }
+          if constexpr (kSplit == 2) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           bool resc = false;
           float alpha = 1.f;
           if (mx > m + kRescaleThreshold) {
@@ -340,25 +355,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float base = (m == -INFINITY) ? 0.f : m;
           float sum = 0.f;
-          uint32_t pk[32];
+          uint32_t pk[kKeys / 2];
 #pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
+          for (int c2 = 0; c2 < kKeys / 2; ++c2) {
             const float p0 = ex2(x[2 * c2] - base);
             const float p1 = ex2(x[2 * c2 + 1] - base);
             sum += p0 + p1;
             pk[c2] = pack2<kBF16>(p0, p1);
           }
-          l = l * alpha + sum;
+          l = l * alpha + sum;  // this lane's keys of the row
           const bool any_resc = __any_sync(0xffffffffu, resc);
-          if (r < NP) s_alpha[b * NP + r] = alpha;
+          if (half == 0 && row < NP) s_alpha[b * NP + row] = alpha;
           if (lane == 0) s_flag[b] = any_resc ? 1 : 0;
           mbar_wait(bar(kPEmpty + b), ((itc >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
-          if (r < NP) {
-            // P row r: 64 keys = 128 bytes, 16-byte chunks XOR-swizzled by row (128-byte swizzle)
-            uint8_t* prow = smem + Lay::kOffP + b * Lay::kPBytes + r * 128;
+          if (row < NP) {
+            // P row: 64 keys = 128 bytes, 16-byte chunks XOR-swizzled by row (128-byte swizzle);
+            // this lane's keys are chunks (kKeys / 8) * half ..
+            uint8_t* prow = smem + Lay::kOffP + b * Lay::kPBytes + row * 128;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              *reinterpret_cast<uint4*>(prow + ((k ^ (r & 7)) << 4)) =
+            for (int k = 0; k < kKeys / 8; ++k)
+              *reinterpret_cast<uint4*>(prow + ((((kKeys / 8) * half + k) ^ (row & 7)) << 4)) =
                   make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
           }
           fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
@@ -395,9 +411,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // be reading it (with one buffer the MMA order already guarantees it finished)
         if (kOBufs == 2 && chunk >= 2)
           mbar_wait(bar(kOEmpty + par), ((chunk >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
-        if (r < NP) {
-          s_lsum[par * NP + r] = l;
-          s_mref[par * NP + r] = m;
+        float lrow = l;
+        if constexpr (kSplit == 2) lrow += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (half == 0 && row < NP) {
+          s_lsum[par * NP + row] = lrow;
+          s_mref[par * NP + row] = m;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kStats + par));
@@ -419,15 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(bar(kQEmpty + (idx & 1)), ((idx >> 1) & 1) ^ 1, wctl, err, kDevErrTimeout);
       __syncwarp();
       tc_fence_after();
+      // with 16 rows, lanes r and r + 16 both hold row r (see the softmax)
+      const int qr = NP == 16 ? (r & 15) : r;
       const uint4* qrow = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint16_t*>(qptr) + (static_cast<int64_t>(c.req) * R + (r < R ? r : 0)) * kDK);
+          reinterpret_cast<const uint16_t*>(qptr) + (static_cast<int64_t>(c.req) * R + (qr < R ? qr : 0)) * kDK);
 #pragma unroll 1
       for (int c32 = 0; c32 < kQCols / 32; ++c32) {
         uint32_t w[32];
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           uint4 d = make_uint4(0, 0, 0, 0);
-          if (r < R) d = __ldg(qrow + c32 * 8 + v);
+          if (qr < R) d = __ldg(qrow + c32 * 8 + v);
           w[4 * v] = d.x;
           w[4 * v + 1] = d.y;
           w[4 * v + 2] = d.z;
