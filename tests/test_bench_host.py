@@ -93,3 +93,25 @@ def test_binding_roof_picks_the_slower_roof():
     assert b == "tensor" and abs(t - 0.01) < 1e-12
     t, b = bench.binding_roof({"bytes": 2e10, "flops": 1e12}, peaks)
     assert b == "hbm" and abs(t - 0.02) < 1e-12
+
+
+def test_fp8_workload_host_logic():
+    """The e5m2-cache workload: its kernel, a cost model at one byte per cached value, and the FP8
+    oracle for the CPU leg."""
+    import torch
+
+    import oracle
+    from workloads import make_case
+
+    assert bench.kernel_of(16, kv_fp8=True) == ("splitkv_fp8_kernel", "splitkv_fp8.cu")
+    assert bench.kernel_of(1024, "row-tile-pair", kv_fp8=True)[0] == "splitkv_fp8_kernel"
+    assert WORKLOADS["memory-bound-fp8"].kv_fp8 and not WORKLOADS["memory-bound"].kv_fp8
+    assert "memory-bound-fp8" in bench.COMPANIONS
+    inp8 = make_case(2, 1, 16, [100, 64], seed=3, kv_fp8=True)
+    inp16 = make_case(2, 1, 16, [100, 64], seed=3)
+    assert inp8.kcache.dtype == torch.uint8
+    c8, c16 = bench.cost_of(inp8, [100, 64]), bench.cost_of(inp16, [100, 64])
+    assert c8["kv_bytes"] == 576 * 164 and c16["kv_bytes"] == 2 * 576 * 164
+    assert c8["flops"] == c16["flops"]
+    assert bench.oracle_fn(inp8) is oracle.mla_decode_fp8_ref
+    assert bench.oracle_fn(inp16) is oracle.mla_decode_ref
