@@ -6,7 +6,8 @@ kernel), inputs resident in HBM.  The headline workload is the memory-bound
 decode batch (64 requests x 4096 cached tokens, h_q 16, s_q 1, bf16); a
 default run adds, under "per_workload", the same measurements for the three
 workloads with h_q * s_q >= 128 (compute-bound, varlen-mtp, long-fp16) and for
-the memory-bound batch over an e5m2 cache (memory-bound-fp8), at most
+the memory- and compute-bound batches over an e5m2 cache (memory-bound-fp8,
+compute-bound-fp8), at most
 --companion-steps timed steps each.  Pick one workload with --workload.
 Throughput uses the pages' cost model: bytes = 576*e*sum(L) + q + out + lse
 (e = 2 bytes per cached value, 1 for the e5m2 cache), FLOPs =
@@ -170,13 +171,15 @@ def variant_of(rows: int, variant: str = "auto") -> str:
     return "few-rows-one-cta" if rows <= 32 else "row-tile-pair"
 
 
-FP8_KERNEL = ("splitkv_fp8_kernel", "splitkv_fp8.cu")
+FP8_KERNELS = (("splitkv_fp8_kernel", "splitkv_fp8.cu"), ("splitkv_fp8_rt_kernel", "splitkv_fp8_rt.cu"))
 
 
 def kernel_of(rows: int, variant: str = "auto", kv_fp8: bool = False):
-    """(name, source file) of the split-KV kernel the library runs for s_q * h_q = rows (one kernel
-    takes every row count over an e5m2 cache)."""
-    return FP8_KERNEL if kv_fp8 else KERNELS[variant_of(rows, variant)]
+    """(name, source file) of the split-KV kernel the library runs for s_q * h_q = rows (over an e5m2
+    cache: the one-CTA kernel up to 32 rows, the 128-row-tile kernel above; variants do not apply)."""
+    if kv_fp8:
+        return FP8_KERNELS[0] if rows <= 32 else FP8_KERNELS[1]
+    return KERNELS[variant_of(rows, variant)]
 
 
 def cost_of(inp, lens):
@@ -568,8 +571,8 @@ def run_sweep(args):
 
 
 # workloads whose numbers join the headline line of a default run: the pages' h_q * s_q >= 128
-# configs, and the headline batch over the e5m2 cache
-COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16", "memory-bound-fp8"]
+# configs, and the memory- and compute-bound batches over an e5m2 cache
+COMPANIONS = ["compute-bound", "varlen-mtp", "long-fp16", "memory-bound-fp8", "compute-bound-fp8"]
 
 
 def run_gpu(args, name: str, companions=()):

@@ -80,8 +80,9 @@ typedef enum { MLA_BF16 = 0, MLA_FP16 = 1 } mla_dtype;
  * saturate), forms q.K from the 8-bit values with fp32 accumulation, runs the
  * softmax in fp32, rounds P to fp16 and multiplies it by V widened to fp16
  * (exact).  The append casts each new value to e5m2 the same way.  Kernel
- * variants (mla_set_kernel_variant) do not apply: one kernel takes every row
- * count, in tiles of 32 query rows.
+ * variants (mla_set_kernel_variant) do not apply: up to 32 query rows one CTA
+ * per partition takes them; above that, two CTAs per tile of 128 rows, each
+ * for half of the 512 output values.
  */
 #define MLA_KV_FP8_E5M2 0x100
 
@@ -150,9 +151,9 @@ int mla_get_workspace_size(int batch, int rows, int num_sm_parts, size_t* bytes)
 
 /*
  * mla_get_num_sm_parts for a given dtype argument: with MLA_KV_FP8_E5M2 set,
- * the e5m2-cache kernel runs one CTA per (partition, tile of 32 query rows)
- * and SM, so num_sm_parts = SMs / ceil(rows / 32) (at least 1); without it,
- * the same as mla_get_num_sm_parts.  Any num_sm_parts >= 1 gives correct
+ * the e5m2-cache kernels run one CTA per SM: num_sm_parts = SMs for up to 32
+ * query rows, SMs / (2 * ceil(rows / 128)) above (at least 1); without it, the
+ * same as mla_get_num_sm_parts.  Any num_sm_parts >= 1 gives correct
  * results; this one fills the GPU once.
  */
 int mla_get_num_sm_parts_dtype(int device, int rows, int dtype, int* num_sm_parts);

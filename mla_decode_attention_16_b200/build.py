@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmla_decode.so")
-SOURCES = ["api.cu", "metadata.cu", "splitkv.cu", "splitkv_narrow.cu", "splitkv_npair.cu", "splitkv_fp8.cu", "combine.cu", "append.cu", "static_ws.cu"]
+SOURCES = ["api.cu", "metadata.cu", "splitkv.cu", "splitkv_narrow.cu", "splitkv_npair.cu", "splitkv_fp8.cu", "splitkv_fp8_rt.cu", "combine.cu", "append.cu", "static_ws.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -114,6 +114,10 @@ int ensure_device(int device) {
           break;
         }
       }
+      if (rc == MLA_OK &&
+          (e = cudaFuncSetAttribute(fp8_rt_kernel_ptr(bf == 1), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fp8_rt_smem_bytes())) != cudaSuccess)
+        rc = cuda_fail(e);
     }
     if (rc != MLA_OK) break;
     if ((e = cudaFuncSetAttribute(metadata_kernel_ptr(), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -306,7 +310,8 @@ int splitkv_impl(const void* q, const void* kcache, int64_t num_pages, const int
   if (is_kv8(dtype)) {  // e5m2 cache: 128-column boxes (128-byte swizzle) + the 64 columns 512..575
     if ((rc = encode_3d_k8(&kmap, kcache, num_pages, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK) return rc;
     if ((rc = encode_3d_k8(&krmap, kcache, num_pages, 64, CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK) return rc;
-    e = launch_splitkv_fp8(bf16, q, kmap, krmap, p, stream);
+    e = base.rows <= kNarrowMaxRows ? launch_splitkv_fp8(bf16, q, kmap, krmap, p, stream)
+                                    : launch_splitkv_fp8_rt(bf16, q, kmap, krmap, p, stream);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e);
   }
   const int kernel = kernel_for(base.rows, g_variant.load());
@@ -412,7 +417,9 @@ int mla_get_num_sm_parts_dtype(int device, int rows, int dtype, int* num_sm_part
   if (rows > kMaxRows) return MLA_ERR_UNSUPPORTED;
   int rc = ensure_device(device);
   if (rc != MLA_OK) return rc;
-  const int parts = g_dev[device].sms / fp8_row_tiles(rows);  // one CTA per (partition, 32-row tile) per SM
+  // one CTA per SM: up to 32 rows one per partition, above that two per 128-row tile
+  const int per_part = rows <= kNarrowMaxRows ? 1 : 2 * fp8_rt_tiles(rows);
+  const int parts = g_dev[device].sms / per_part;
   *num_sm_parts = parts > 0 ? parts : 1;
   return MLA_OK;
 }

@@ -34,6 +34,12 @@ int fp8_smem_bytes(int np);
 const void* fp8_kernel_ptr(bool bf16, int np);
 cudaError_t launch_splitkv_fp8(bool bf16, const void* q, const CUtensorMap& kmap, const CUtensorMap& krmap,
                                const DecodeParams& p, cudaStream_t stream);
+// Split-KV kernel over an e5m2 cache for s_q * h_q > 32: two CTAs (value halves) per 128-row tile.
+int fp8_rt_tiles(int rows);
+int fp8_rt_smem_bytes();
+const void* fp8_rt_kernel_ptr(bool bf16);
+cudaError_t launch_splitkv_fp8_rt(bool bf16, const void* q, const CUtensorMap& kmap, const CUtensorMap& krmap,
+                                  const DecodeParams& p, cudaStream_t stream);
 cudaError_t launch_combine(bool bf16, const DecodeParams& p, cudaStream_t stream);
 // Copies kv_new [batch, s_q, 576] into cache positions L_b - s_q + s (programmatic dependent launch).
 cudaError_t launch_append(const void* kv_new, void* kcache, int64_t num_pages, const int32_t* block_table,

@@ -257,6 +257,16 @@ __device__ __forceinline__ void umma_ts_e5m2(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem desc] * B[smem desc] with 8-bit operands (kind::f8f6f4, K = 32 per instruction).
+__device__ __forceinline__ void umma_ss_e5m2(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on `bar` when every tcgen05 async op issued so far by this thread completes.
 // Weight-stationary form (M = 32 / 64 / 128): with M = 32 the D tile of N columns is spread over
 // the four TMEM lane quadrants, quadrant q holding rows 0..31 in its lanes and the columns

@@ -104,7 +104,9 @@ def test_fp8_workload_host_logic():
     from workloads import make_case
 
     assert bench.kernel_of(16, kv_fp8=True) == ("splitkv_fp8_kernel", "splitkv_fp8.cu")
-    assert bench.kernel_of(1024, "row-tile-pair", kv_fp8=True)[0] == "splitkv_fp8_kernel"
+    assert bench.kernel_of(32, kv_fp8=True)[0] == "splitkv_fp8_kernel"
+    assert bench.kernel_of(33, kv_fp8=True) == ("splitkv_fp8_rt_kernel", "splitkv_fp8_rt.cu")
+    assert bench.kernel_of(1024, "row-tile-pair", kv_fp8=True)[0] == "splitkv_fp8_rt_kernel"
     assert WORKLOADS["memory-bound-fp8"].kv_fp8 and not WORKLOADS["memory-bound"].kv_fp8
     assert "memory-bound-fp8" in bench.COMPANIONS
     inp8 = make_case(2, 1, 16, [100, 64], seed=3, kv_fp8=True)

@@ -38,12 +38,13 @@ def _hook(lib, enable, cycles):
     (3, 1, 16, [700, 64, 2000], False, 1, "few-rows-pair"),
     (2, 2, 64, [900, 300], True, 2, "row-tile-pair"),
     (3, 1, 16, [700, 64, 2000], False, 3, "fp8-cache"),
+    (2, 2, 64, [900, 300], True, 4, "fp8-cache-128-row-tiles"),
 ], ids=lambda c: c[-1])
 def test_withheld_arrival_times_out_and_launch_returns(case):
     import mla_decode_attention_16_b200 as mla
 
     b, s_q, h_q, lens, causal, seed, variant = case
-    kv_fp8 = variant == "fp8-cache"  # the e5m2-cache kernel (kernel variants do not apply to it)
+    kv_fp8 = variant.startswith("fp8-cache")  # the e5m2-cache kernels (kernel variants do not apply)
     inp = make_case(b, s_q, h_q, lens, causal=causal, seed=300 + seed, kv_fp8=kv_fp8)
     ref = oracle.mla_decode_fp8_ref if kv_fp8 else oracle.mla_decode_ref
     variant = "auto" if kv_fp8 else variant

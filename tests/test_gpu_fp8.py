@@ -21,16 +21,18 @@ CASES = [
     (3, 1, 16, [1, 63, 200], torch.bfloat16, False, None, 1),         # 16 rows: one tile, NP = 16
     (2, 1, 32, [64, 300], torch.float16, False, None, 2),             # 32 rows: one full tile
     (2, 2, 16, [129, 2], torch.bfloat16, True, None, 3),              # causal, s_q = 2
-    (2, 1, 64, [70, 1000], torch.bfloat16, False, None, 4),           # 2 row tiles
-    (2, 2, 128, [70, 1], torch.bfloat16, True, None, 5),              # 8 row tiles; a row with no visible key
-    (2, 1, 33, [300, 64], torch.float16, False, None, 6),             # ragged second tile of one row
+    (2, 1, 64, [70, 1000], torch.bfloat16, False, None, 4),           # 64 rows: one half-empty tile
+    (2, 2, 128, [70, 1], torch.bfloat16, True, None, 5),              # 2 row tiles; a row with no visible key
+    (2, 1, 33, [300, 64], torch.float16, False, None, 6),             # 33 rows: the 128-row kernel
     (4, 1, 16, [0, 5, 0, 640], torch.bfloat16, False, 3, 7),          # empty requests, splits
     (1, 1, 16, [1000], torch.bfloat16, False, 7, 8),                  # one request cut in many chunks
     (1, 2, 8, [513], torch.float16, True, 1, 9),                      # single partition
     (5, 1, 1, [17, 64, 65, 128, 129], torch.bfloat16, False, 2, 10),  # one query row
     (600, 1, 16, [(37 * i) % 211 for i in range(600)], torch.bfloat16, False, None, 11),  # many short requests
-    (1, 8, 128, [700], torch.bfloat16, True, None, 12),               # 1024 rows: 32 row tiles
-    (4, 1, 64, [0, 5, 0, 640], torch.float16, False, 3, 13),          # row tiles with splits
+    (1, 8, 128, [700], torch.bfloat16, True, None, 12),               # 1024 rows: 8 row tiles
+    (4, 1, 64, [0, 5, 0, 640], torch.float16, False, 3, 13),          # 128-row kernel with splits
+    (3, 1, 128, [4096, 70, 1], torch.bfloat16, False, None, 14),      # one full 128-row tile, long request
+    (2, 2, 100, [300, 77], torch.float16, True, None, 15),            # 200 rows: a ragged second tile
 ]
 
 
@@ -143,5 +145,16 @@ def test_fp8_partition_count():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert mla.mla_get_num_sm_parts(16, kv_fp8=True) == sms
     assert mla.mla_get_num_sm_parts(32, kv_fp8=True) == sms
-    assert mla.mla_get_num_sm_parts(128, kv_fp8=True) == sms // 4
-    assert mla.mla_get_num_sm_parts(1024, kv_fp8=True) == sms // 32
+    assert mla.mla_get_num_sm_parts(33, kv_fp8=True) == sms // 2   # one 128-row tile, two CTAs
+    assert mla.mla_get_num_sm_parts(128, kv_fp8=True) == sms // 2
+    assert mla.mla_get_num_sm_parts(1024, kv_fp8=True) == sms // 16
+
+
+def test_fp8_cache_compute_bound_workload_every_request():
+    """The full-size e5m2 workload with 128 query rows (128 requests x 4096 tokens), every request
+    checked: the 128-row-tile kernel."""
+    inp = make_workload("compute-bound-fp8")
+    out, lse, _, _, flags = run_gpu(inp)
+    assert flags[0] == 0
+    ref_out, ref_lse = _ref(inp)
+    compare(out, lse, ref_out, ref_lse, "compute-bound-fp8")

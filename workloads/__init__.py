@@ -19,7 +19,8 @@ varlen-mtp      132    2   128  uniform int in [1,16384] bf16    1.0        yes
 long-fp16        16    2    64  32768 + uniform [-2048,2048] fp16 0.5       yes
 =============== ===== ==== ==== ======================== ======= ========== ======
 
-``memory-bound-fp8`` is ``memory-bound`` with an e5m2 cache (one byte per value).  An e5m2
+``memory-bound-fp8`` / ``compute-bound-fp8`` are ``memory-bound`` / ``compute-bound`` with an
+e5m2 cache (one byte per value).  An e5m2
 cache is drawn as raw codes (no rounding of any number happens here): sign and 2-bit mantissa
 uniform, exponent field uniform in [10, 16] (magnitudes 2^-5 .. 3.5, a spread like the 16-bit
 caches' N(0, 1)); its poison is code 0x71 (10240).
@@ -78,6 +79,8 @@ WORKLOADS: Dict[str, Workload] = {
                  description="batch 64, s_q 1, h_q 16, seqlen 4096, bf16"),
         Workload("memory-bound-fp8", 64, 1, 16, torch.bfloat16, 1.0, False, 1005, "fixed", 4096,
                  description="batch 64, s_q 1, h_q 16, seqlen 4096, bf16 q, e5m2 cache", kv_fp8=True),
+        Workload("compute-bound-fp8", 128, 1, 128, torch.bfloat16, 1.0, False, 1006, "fixed", 4096,
+                 description="batch 128, s_q 1, h_q 128, seqlen 4096, bf16 q, e5m2 cache", kv_fp8=True),
         Workload("compute-bound", 128, 1, 128, torch.bfloat16, 1.0, False, 1002, "fixed", 4096,
                  description="batch 128, s_q 1, h_q 128, seqlen 4096, bf16"),
         Workload("varlen-mtp", 132, 2, 128, torch.bfloat16, 1.0, True, 1003, "uniform", 1, 16384,
