@@ -182,6 +182,18 @@ def kernel_of(rows: int, variant: str = "auto", kv_fp8: bool = False):
     return KERNELS[variant_of(rows, variant)]
 
 
+def tensor_peak(peaks: dict, kv_fp8: bool) -> float:
+    """Tensor-core peak (TF/s) a decode's FLOPs are held to.  16-bit: the measured bf16 rate (fp16
+    runs at the same dense rate).  e5m2 cache: Q.K^T (576 of the 1088 FLOPs per key and row) runs
+    as an 8-bit MMA at twice that rate (the nominal fp8 : bf16 ratio), P.V at the 16-bit rate, so
+    the peak is the FLOP-weighted harmonic blend of the two."""
+    bf16 = float(peaks["bf16_tflops"])
+    if not kv_fp8:
+        return bf16
+    f_qk, f_pv = 576.0, 512.0
+    return (f_qk + f_pv) / (f_qk / (2.0 * bf16) + f_pv / bf16)
+
+
 def cost_of(inp, lens):
     """The pages' cost model for these requests of a workload (1 byte per value of an e5m2 cache)."""
     return algorithmic_cost(lens, inp.s_q, inp.h_q, kv_elem_bytes=inp.kcache.element_size())
@@ -458,7 +470,7 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak}
     else:
         achieved = cost["flops"] / kern_s / 1e12
-        peak = float(peaks["bf16_tflops"])  # fp16 dense tensor rate equals bf16 on this part
+        peak = tensor_peak(peaks, w.kv_fp8)
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
     kname, ksrc = kernel_of(rows, variant, w.kv_fp8)
     roof["traffic"] = profile_traffic(name, kname, ksrc)

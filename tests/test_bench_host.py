@@ -117,3 +117,12 @@ def test_fp8_workload_host_logic():
     assert c8["flops"] == c16["flops"]
     assert bench.oracle_fn(inp8) is oracle.mla_decode_fp8_ref
     assert bench.oracle_fn(inp16) is oracle.mla_decode_ref
+
+
+def test_tensor_peak_blends_fp8_and_fp16():
+    """Over an e5m2 cache Q.K^T (576 of 1088 FLOPs per key) runs at twice the 16-bit rate."""
+    peaks = {"bf16_tflops": 1000.0}
+    assert bench.tensor_peak(peaks, False) == 1000.0
+    blended = bench.tensor_peak(peaks, True)
+    assert abs(blended - 1088.0 / (576.0 / 2000.0 + 512.0 / 1000.0)) < 1e-9
+    assert 1000.0 < blended < 2000.0
