@@ -156,7 +156,6 @@ def mla_decode_fp8_ref(
         raise ValueError("kcache_codes must hold uint8 e5m2 codes")
     b, s_q, h_q, _ = q.shape
     reqs = list(range(b)) if requests is None else [int(r) for r in requests]
-    q8 = e5m2_quantize(q.to(_F64))
     out = torch.zeros(len(reqs), s_q, h_q, 512, dtype=_F64)
     lse = torch.full((len(reqs), h_q, s_q), -math.inf, dtype=_F64)
     for i, r in enumerate(reqs):
@@ -166,7 +165,8 @@ def mla_decode_fp8_ref(
         pages = block_table[r, :n].to(torch.int64)
         k8 = e5m2_decode(kcache_codes[pages])
         table = torch.arange(max(n, 1), dtype=torch.int32)[None]
-        o, l = mla_decode_ref(q8[r:r + 1], k8.reshape(n, 64, 1, 576), table, cache_seqlens[r:r + 1],
+        q8 = e5m2_quantize(q[r:r + 1].to(_F64))  # this request's query rows cast to e5m2
+        o, l = mla_decode_ref(q8, k8.reshape(n, 64, 1, 576), table, cache_seqlens[r:r + 1],
                               softmax_scale, causal)
         out[i] = o[0]
         lse[i] = l[0]

@@ -85,7 +85,7 @@ FP8_MUTANTS = {
     "subnormals one binade low": ("return sign * (m / 4.0) * 2.0 ** E5M2_MIN_NORMAL_EXP",
                                   "return sign * (m / 4.0) * 2.0 ** (E5M2_MIN_NORMAL_EXP - 1)"),
     "mantissa bits swapped": ("m = code & 0x3", "m = ((code & 1) << 1) | ((code >> 1) & 1)"),
-    "query not cast": ("q8 = e5m2_quantize(q.to(_F64))", "q8 = q.to(_F64)"),
+    "query not cast": ("q8 = e5m2_quantize(q[r:r + 1].to(_F64))", "q8 = q[r:r + 1].to(_F64)"),
     "append stores truncated bytes": ("e5m2_encode(kv_new.to(_F64)))", "kv_new.to(torch.uint8))"),
     "sign dropped": ("out = torch.where(finite_nz, torch.copysign(q, x), x)", "out = torch.where(finite_nz, q, x)"),
 }
