@@ -26,15 +26,17 @@
 // (the Q.K^T MMA computes all 128 lanes; rows outside the current quadrant are
 // ignored).
 //
-// Roles (384 threads): warp 0 lane 0 TMA producer; warp 1 TMEM owner, lane 0
-// issues the Q.K^T MMAs; warps 4-7: warp 4 + (chunk & 1) runs the softmax of a
-// chunk (one thread per query row), all four rescale O when a row's exponent
-// reference moves, and warp 6 lane 0 issues the P.V MMAs; warps 8-11 write each
-// chunk's epilogue, and warps 8 / 9 load Q for even / odd chunks.  With one
-// thread issuing both products, a page's P.V had to wait behind the next page's
-// Q.K^T, holding the page's 72 KB stage that much longer; with two issuers P.V
-// goes as soon as P is written (tcgen05.commit tracks the issuing thread's own
-// MMAs, so each issuer commits its own barriers).
+// Roles (384 threads): warp 0 lane 0 issues the page loads and the P.V MMAs,
+// whichever is ready first; warp 1 TMEM owner, lane 0 issues the Q.K^T MMAs;
+// warps 4-7: warp 4 + (chunk & 1) runs the softmax of a chunk (one thread per
+// query row), all four rescale O when a row's exponent reference moves; warps
+// 8-11 write each chunk's epilogue, and warps 8 / 9 load Q for even / odd
+// chunks.  With one thread issuing both products, a page's P.V had to wait
+// behind the next page's Q.K^T, holding the page's 72 KB stage that much
+// longer; with P.V on its own issuer it goes as soon as P is written
+// (tcgen05.commit tracks the issuing thread's own MMAs, so each issuer commits
+// its own barriers).  The load thread polls both queues without blocking, so a
+// free stage is refilled at once and no softmax warp stalls to issue MMAs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* err = p.err;
 
   // O[:, 256h ..] += P[:, 16kk ..] . V[16kk .., 256h ..] for page itp (chunk-relative index jjp of
-  // chunk `chunk`), issued by warp 6 lane 0 once the four softmax warps have released P.  A = P (32
+  // chunk `chunk`), issued by the load thread once the four softmax warps have released P.  A = P (32
   // rows, K-major), B = V (MN-major view of the page's column boxes 4h .. 4h+3, 8 KB apart; 16 keys
   // = 2 x 1 KB).  Its commit also frees the page stage: the page's Q.K^T, issued by the other
   // thread, completed before its softmax could write P.
@@ -208,37 +210,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (pages only)
+    // ------------------------------------------------------------ page loads and P.V issue
     if (lane == 0) {
       const uint64_t evict_first = policy_evict_first();
-      uint32_t it = 0;
-      int cur = br;
-      Chunk ch;
-      while (!aborted(wctl) && next_chunk(p, br, bk, er, ek, bs, cur, ch)) {
-        const int32_t* bt = p.block_table + static_cast<int64_t>(ch.req) * p.block_table_stride;
-        int page_next = bt[ch.lo];
-        for (int blk = ch.lo; blk < ch.hi; ++blk, ++it) {
-          if (aborted(wctl)) break;
-          const int st = it % kStages;
-          int page = page_next;
-          if (blk + 1 < ch.hi) page_next = bt[blk + 1];  // read while this stage frees up
-          if (!mbar_wait(bar(kKvEmpty + st), ((it / kStages) & 1) ^ 1, wctl, err, kDevErrTimeout)) break;
-          if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
-            atomicOr(err, kDevErrPage);
-            atomicCAS(err + 1, 0, page == 0 ? -1 : page);
-            page = 0;
-          }
-          mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
-          for (int i = 0; i < kBoxes; ++i)
-            tma_load_3d_hint(sbase + Lay::kOffK + st * kStageBytes + i * kKBox, &kmap, bar(kKvFull + st), 64 * i,
-                             0, page, evict_first);
+      Walk wl, wp;
+      wl.init(p, meta);
+      wp = wl;
+      uint32_t tl = 0, tp = 0;
+      auto pv_ready = [&]() {
+        if (wp.first() && !mbar_test_wait(bar(kOEmpty), (wp.chunk & 1) ^ 1)) return false;
+        return mbar_test_wait(bar(kPFull + (tp & 1)), (tp >> 1) & 1);
+      };
+      auto issue_load = [&]() {
+        const int st = tl % kStages;
+        int page = p.block_table[static_cast<int64_t>(wl.req) * p.block_table_stride + wl.blk];
+        if (page < 0 || static_cast<int64_t>(page) >= p.num_pages) {
+          atomicOr(err, kDevErrPage);
+          atomicCAS(err + 1, 0, page == 0 ? -1 : page);
+          page = 0;
         }
+        mbar_arrive_expect_tx(bar(kKvFull + st), kStageBytes);
+        for (int i = 0; i < kBoxes; ++i)
+          tma_load_3d_hint(sbase + Lay::kOffK + st * kStageBytes + i * kKBox, &kmap, bar(kKvFull + st), 64 * i, 0,
+                           page, evict_first);
+        wl.next(p);
+        ++tl;
+      };
+      long long idle_since = clock64();
+      uint32_t polls = 0;
+      while (wp.valid) {
+        if (wl.valid && mbar_test_wait(bar(kKvEmpty + tl % kStages), ((tl / kStages) & 1) ^ 1)) {
+          issue_load();
+        } else if (tp < tl && pv_ready()) {
+          issue_pv(tp, wp.first() ? 0 : 1, wp.last(), static_cast<uint32_t>(wp.chunk));
+          wp.next(p);
+          ++tp;
+        } else {
+          if ((++polls & 15u) == 0) {
+            if (aborted(wctl)) break;
+            if (clock64() - idle_since > wctl->limit) {
+              raise_abort(wctl);
+              atomicOr(err, kDevErrTimeout);
+              break;
+            }
+          }
+          continue;
+        }
+        idle_since = clock64();
       }
-      // Before the CTA can exit, every page load issued above must have landed: wait (bounded, abort
-      // or not) for the last phase of each stage.  A phase the MMA warp already consumed has
-      // completed, so the wait returns at once; only an abort leaves one pending.
-      for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+      // Before the CTA can exit, every page load issued above must have landed and every P.V
+      // issued here must have completed: bounded waits, abort or not (a phase already consumed
+      // has completed, so the wait returns at once; only an abort leaves one pending).
+      for (uint32_t j = tl > kStages ? tl - kStages : 0; j < tl; ++j)
         mbar_wait_drain(bar(kKvFull + j % kStages), (j / kStages) & 1, wctl->limit);
+      umma_commit(bar(kDrainPV));
+      mbar_wait_drain(bar(kDrainPV), 0, wctl->limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ Q.K^T issuer
@@ -401,10 +427,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kPFull + b));
-        if (warp == 6) {  // this page's P.V (after all four warps arrived: P written, O rescaled)
-          if (lane == 0 && !aborted(wctl)) issue_pv(itc, jj, jj == nb - 1, chunk);
-          __syncwarp();
-        }
       }
       if (smx) {
         // this stats slot was last used by chunk - 2; with two O buffers its epilogue may still
@@ -422,10 +444,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       it += nb;
       ++chunk;
-    }
-    if (warp == 6 && lane == 0) {
-      umma_commit(bar(kDrainPV));
-      mbar_wait_drain(bar(kDrainPV), 0, wctl->limit);
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------ Q loads (warps 8 / 9) and epilogue (8-11)
