@@ -182,16 +182,59 @@ def kernel_of(rows: int, variant: str = "auto", kv_fp8: bool = False):
     return KERNELS[variant_of(rows, variant)]
 
 
-def tensor_peak(peaks: dict, kv_fp8: bool) -> float:
+# Context denominators besides the measured ones: the ~8 TB/s HBM figure the target states, and
+# the datasheet dense bf16 rate of one B200.
+NOMINAL_HBM_GBS = 8000.0
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def tensor_peak(peaks: dict, kv_fp8: bool, key: str = "bf16_tflops") -> float:
     """Tensor-core peak (TF/s) a decode's FLOPs are held to.  16-bit: the measured bf16 rate (fp16
     runs at the same dense rate).  e5m2 cache: Q.K^T (576 of the 1088 FLOPs per key and row) runs
     as an 8-bit MMA at twice that rate (the nominal fp8 : bf16 ratio), P.V at the 16-bit rate, so
-    the peak is the FLOP-weighted harmonic blend of the two."""
-    bf16 = float(peaks["bf16_tflops"])
+    the peak is the FLOP-weighted harmonic blend of the two.  `key` picks the bf16 rate."""
+    bf16 = float(peaks[key])
     if not kv_fp8:
         return bf16
     f_qk, f_pv = 576.0, 512.0
     return (f_qk + f_pv) / (f_qk / (2.0 * bf16) + f_pv / bf16)
+
+
+def roofline_extras(unit: str, achieved: float, peaks: dict, kv_fp8: bool, read_gbs) -> dict:
+    """The same achieved rate against the other denominators: for HBM-bound work the nominal
+    8 TB/s and a read-only stream measured in the same run; for tensor-bound work the sustained
+    (seconds-long, power-capped) bf16 rate and the datasheet rate, blended like the primary peak
+    for an e5m2 cache."""
+    if unit == "GB/s":
+        return {"nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                "read_stream_gbs": read_gbs, "frac_of_read_stream": achieved / read_gbs if read_gbs else None}
+    sustained = tensor_peak(peaks, kv_fp8, "bf16_tflops_sustained")
+    nominal = tensor_peak({"bf16_tflops": NOMINAL_BF16_TFLOPS}, kv_fp8)
+    return {"sustained_peak": sustained, "frac_of_sustained": achieved / sustained,
+            "nominal_peak": nominal, "frac_of_nominal": achieved / nominal}
+
+
+_READ_STREAM = {}
+
+
+def read_stream_gbs(dev) -> float:
+    """Read-only HBM stream of this GPU, measured once per process: a sum over 2 GiB of bf16
+    (larger than L2), best of 5, CUDA events.  A denominator for context only (a library kernel,
+    outside every timed region)."""
+    if dev.index not in _READ_STREAM:
+        x = torch.ones(1 << 30, dtype=torch.bfloat16, device=dev)
+        best = float("inf")
+        for _ in range(6):
+            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            x.sum(dtype=torch.float32)
+            z.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, a.elapsed_time(z) / 1000.0)
+        _READ_STREAM[dev.index] = x.numel() * x.element_size() / best / 1e9
+        del x
+        torch.cuda.empty_cache()
+    return _READ_STREAM[dev.index]
 
 
 def cost_of(inp, lens):
@@ -480,6 +523,7 @@ def measure_gpu(name: str, steps: int, warmup: int, world: int, rank: int, dev, 
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak}
     kname, ksrc = kernel_of(rows, variant, w.kv_fp8)
     roof["traffic"] = profile_traffic(name, kname, ksrc)
+    roof.update(roofline_extras(unit, achieved, peaks, w.kv_fp8, read_stream_gbs(dev) if unit == "GB/s" else None))
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["kernel"] = kname
     roof["variant"] = "fp8-cache" if w.kv_fp8 else variant_of(rows, variant)

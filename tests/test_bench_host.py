@@ -126,3 +126,19 @@ def test_tensor_peak_blends_fp8_and_fp16():
     blended = bench.tensor_peak(peaks, True)
     assert abs(blended - 1088.0 / (576.0 / 2000.0 + 512.0 / 1000.0)) < 1e-9
     assert 1000.0 < blended < 2000.0
+
+
+def test_roofline_extras_denominators():
+    """HBM-bound work is also held to the nominal 8 TB/s and to a read stream of the same run;
+    tensor-bound work to the sustained and datasheet bf16 rates, blended for an e5m2 cache like
+    the primary peak."""
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    h = bench.roofline_extras("GB/s", 4000.0, peaks, False, 6400.0)
+    assert h["frac_of_nominal"] == 0.5 and h["frac_of_read_stream"] == 0.625
+    assert bench.roofline_extras("GB/s", 4000.0, peaks, False, None)["frac_of_read_stream"] is None
+    t = bench.roofline_extras("TFLOPS", 700.0, peaks, False, None)
+    assert t["sustained_peak"] == 1400.0 and t["frac_of_sustained"] == 0.5
+    assert t["nominal_peak"] == 2250.0
+    t8 = bench.roofline_extras("TFLOPS", 700.0, peaks, True, None)
+    assert abs(t8["sustained_peak"] - bench.tensor_peak({"bf16_tflops": 1400.0}, True)) < 1e-9
+    assert abs(t8["nominal_peak"] - bench.tensor_peak({"bf16_tflops": 2250.0}, True)) < 1e-9
