@@ -218,7 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       wp = wl;
       uint32_t tl = 0, tp = 0;
       auto pv_ready = [&]() {
-        if (wp.first() && !mbar_test_wait(bar(kOEmpty), (wp.chunk & 1) ^ 1)) return false;
+        // the same O-buffer phase that issue_pv waits for
+        if (wp.first() && !mbar_test_wait(bar(kOEmpty + wp.chunk % kOBufs), ((wp.chunk / kOBufs) & 1) ^ 1))
+          return false;
         return mbar_test_wait(bar(kPFull + (tp & 1)), (tp >> 1) & 1);
       };
       auto issue_load = [&]() {
